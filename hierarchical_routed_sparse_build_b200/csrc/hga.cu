@@ -1,0 +1,344 @@
+// libhga: C ABI entry points (include/hga.h) for routed attention on sm_100a.
+//
+// Host code validates every argument before anything is enqueued, picks the
+// launch shape, and launches the kernels of hga_summaries.cuh and
+// hga_routed.cuh on the caller's stream. No device memory is allocated here.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "hga.h"
+#include "hga_common.cuh"
+#include "hga_routed.cuh"
+#include "hga_summaries.cuh"
+
+namespace hga {
+namespace {
+
+std::atomic<int> g_ctas_per_head{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hga_status check_kv(const hga_kv* kv, bool need_v) {
+  if (kv == nullptr || kv->k == nullptr || kv->seq_lens == nullptr) return HGA_ERR_INVALID_ARG;
+  if (need_v && kv->v == nullptr) return HGA_ERR_INVALID_ARG;
+  if (kv->batch < 1 || kv->n_kv_heads < 1 || kv->max_len < 1 || kv->head_dim < 1)
+    return HGA_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+  if (!aligned16(kv->k) || (need_v && !aligned16(kv->v))) return HGA_ERR_INVALID_ARG;
+  if (kv->page_table != nullptr) {
+    if (kv->page_size < 1 || kv->max_pages < 1 || kv->num_pages < 1) return HGA_ERR_INVALID_ARG;
+    if ((int64_t)kv->max_pages * kv->page_size < kv->max_len) return HGA_ERR_INVALID_ARG;
+    if ((int64_t)kv->num_pages * kv->n_kv_heads * kv->page_size >= (int64_t)UINT32_MAX)
+      return HGA_ERR_UNSUPPORTED;
+  } else {
+    if ((int64_t)kv->batch * kv->n_kv_heads * kv->max_len >= (int64_t)UINT32_MAX)
+      return HGA_ERR_UNSUPPORTED;
+  }
+  return HGA_OK;
+}
+
+hga_status check_params(const hga_params* p, const hga_kv* kv, bool routing) {
+  if (p == nullptr) return HGA_ERR_INVALID_ARG;
+  if (!(p->scale >= 0.f) || std::isinf(p->scale)) return HGA_ERR_INVALID_ARG;
+  if (!routing) return HGA_OK;
+  if (p->chunk < 1 || p->group < 1 || p->chunk % p->group != 0) return HGA_ERR_INVALID_ARG;
+  if (p->top_chunks < 1 || p->top_groups < 1 || p->top_groups > p->chunk / p->group)
+    return HGA_ERR_INVALID_ARG;
+  if (p->chunk / p->group > kMaxGroupsPerChunk) return HGA_ERR_UNSUPPORTED;
+  if (kv->max_len / p->chunk > kMaxChunks) return HGA_ERR_UNSUPPORTED;
+  if (kv->page_table != nullptr && kv->page_size != p->chunk) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+hga_status check_heads(int32_t n_q_heads, const hga_kv* kv) {
+  if (n_q_heads < 1 || n_q_heads % kv->n_kv_heads != 0) return HGA_ERR_INVALID_ARG;
+  if (n_q_heads / kv->n_kv_heads > kMaxHeadsPerKv) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+int max_routed(const hga_kv* kv, const hga_params* p) {
+  const int C = p->chunk, g = p->group, gk = p->top_groups;
+  const int nf_max = kv->max_len / C;
+  int best = kv->max_len < 3 * C - 1 ? kv->max_len : 3 * C - 1;  // nf <= 2: dense
+  for (int nf = 3; nf <= nf_max; ++nf) {
+    const int r = nf - 2 < p->top_chunks ? nf - 2 : p->top_chunks;
+    const int tail = kv->max_len - nf * C < C - 1 ? kv->max_len - nf * C : C - 1;
+    const int s = 2 * C + r * gk * g + tail;
+    if (s > best) best = s;
+  }
+  return best;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+int pick_cluster(int units) {
+  int P = g_ctas_per_head.load();
+  if (P > 0) return P;
+  // about two co-resident CTAs per SM in total, at most 8 per (sequence, KV head)
+  P = (2 * sm_count() + units - 1) / units;
+  return P < 1 ? 1 : (P > 8 ? 8 : P);
+}
+
+KvView make_kv_view(const hga_kv* kv) {
+  KvView v;
+  v.k = static_cast<const uint16_t*>(kv->k);
+  v.v = static_cast<const uint16_t*>(kv->v);
+  v.page_table = kv->page_table;
+  v.seq_lens = kv->seq_lens;
+  v.batch = kv->batch;
+  v.hkv = kv->n_kv_heads;
+  v.max_len = kv->max_len;
+  v.page_size = kv->page_table ? kv->page_size : 0;
+  v.max_pages = kv->page_table ? kv->max_pages : 0;
+  v.num_pages = kv->page_table ? kv->num_pages : 0;
+  return v;
+}
+
+SumView make_sum_view(const hga_kv* kv, const hga_params* p, const void* cs, const void* gs) {
+  SumView s;
+  s.chunk = const_cast<uint16_t*>(static_cast<const uint16_t*>(cs));
+  s.group = const_cast<uint16_t*>(static_cast<const uint16_t*>(gs));
+  s.max_chunks = p ? kv->max_len / p->chunk : 0;
+  s.gpc = p ? p->chunk / p->group : 1;
+  s.d = kv->head_dim;
+  return s;
+}
+
+float scale_log2(const hga_params* p, int d) {
+  const double sc = p->scale > 0.f ? (double)p->scale : 1.0 / std::sqrt((double)d);
+  return (float)(sc * 1.4426950408889634074);
+}
+
+template <int D, int MODE>
+cudaError_t launch_routed(const RoutedArgs& a, int units, int P, cudaStream_t stream) {
+  const RoutedSmem lay(D, a.n_pad, a.kcap, a.G);
+  auto kern = routed_kernel<D, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+  if (e != cudaSuccess) return e;
+  if (P > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3((unsigned)(units * P), 1, 1);
+  cfg.blockDim = dim3(kRoutedThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)lay.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int MODE>
+hga_status run_routed(RoutedArgs a, int D, int units, cudaStream_t stream) {
+  const int P = pick_cluster(units);
+  cudaError_t e = D == 128 ? launch_routed<128, MODE>(a, units, P, stream)
+                           : launch_routed<64, MODE>(a, units, P, stream);
+  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+int next_pow2(int x) {
+  int p = 2;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// Fill the routing part of RoutedArgs (n_pad, kcap, params).
+void routing_args(RoutedArgs& a, const hga_kv* kv, const hga_params* p) {
+  const int nf_max = kv->max_len / p->chunk;
+  const int cand_max = nf_max > 2 ? nf_max - 2 : 0;
+  a.C = p->chunk;
+  a.g = p->group;
+  a.k = p->top_chunks;
+  a.G = p->top_groups;
+  a.n_pad = next_pow2(cand_max);
+  const int kc = cand_max < p->top_chunks ? cand_max : p->top_chunks;
+  a.kcap = kc < 1 ? 1 : kc;
+}
+
+}  // namespace
+}  // namespace hga
+
+using namespace hga;
+
+extern "C" {
+
+const char* hga_status_string(hga_status s) {
+  switch (s) {
+    case HGA_OK: return "ok";
+    case HGA_ERR_INVALID_ARG: return "invalid argument";
+    case HGA_ERR_UNSUPPORTED: return "unsupported size or layout";
+    case HGA_ERR_CUDA: return "CUDA runtime error";
+    case HGA_ERR_DEVICE_FAULT: return "bad device-side input (skipped by the kernel)";
+    case HGA_ERR_TIMEOUT: return "bounded device wait expired";
+  }
+  return "unknown status";
+}
+
+hga_status hga_summary_bytes(const hga_kv* kv, const hga_params* p, size_t* chunk_bytes,
+                             size_t* group_bytes) {
+  hga_status s = check_kv(kv, false);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  const size_t d = (size_t)kv->head_dim, gpc = (size_t)(p->chunk / p->group);
+  const size_t slots = kv->page_table ? (size_t)kv->num_pages * kv->n_kv_heads
+                                      : (size_t)kv->batch * kv->n_kv_heads * (kv->max_len / p->chunk);
+  if (chunk_bytes) *chunk_bytes = slots * d * 2;
+  if (group_bytes) *group_bytes = slots * gpc * d * 2;
+  return HGA_OK;
+}
+
+int32_t hga_max_routed_tokens(const hga_kv* kv, const hga_params* p) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK) return -1;
+  return max_routed(kv, p);
+}
+
+hga_status hga_build_summaries(const hga_kv* kv, const hga_params* p, void* chunk_sum,
+                               void* group_sum, cudaStream_t stream) {
+  hga_status s = check_kv(kv, false);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum))
+    return HGA_ERR_INVALID_ARG;
+  const int max_chunks = kv->max_len / p->chunk;
+  if (max_chunks == 0) return HGA_OK;
+  const int gpc = p->chunk / p->group;
+  const KvView kvv = make_kv_view(kv);
+  const SumView sv = make_sum_view(kv, p, chunk_sum, group_sum);
+  dim3 grid((unsigned)max_chunks, (unsigned)kv->n_kv_heads, (unsigned)kv->batch);
+  dim3 block((unsigned)(32 * (gpc < 8 ? gpc : 8)));
+  const size_t smem = (size_t)gpc * kv->head_dim * sizeof(float);
+  if (kv->head_dim == 128)
+    summaries_kernel<128><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group);
+  else
+    summaries_kernel<64><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group);
+  return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+hga_status hga_route(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                     const void* group_sum, const hga_params* p, int32_t* idx, int32_t idx_stride,
+                     int32_t* n_idx, cudaStream_t stream) {
+  hga_status s = check_kv(kv, false);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || group_sum == nullptr ||
+      !aligned16(chunk_sum) || !aligned16(group_sum) || idx == nullptr || n_idx == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if (idx_stride < max_routed(kv, p)) return HGA_ERR_INVALID_ARG;
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.kv = make_kv_view(kv);
+  a.sv = make_sum_view(kv, p, chunk_sum, group_sum);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  routing_args(a, kv, p);
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.idx_out = idx;
+  a.n_idx_out = n_idx;
+  a.idx_stride = idx_stride;
+  return run_routed<kModeRoute>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+hga_status hga_attend(const void* q, int32_t n_q_heads, const hga_kv* kv, const int32_t* idx,
+                      int32_t idx_stride, const int32_t* n_idx, const hga_params* p, float* out,
+                      float* lse, cudaStream_t stream) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, false)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || idx == nullptr || n_idx == nullptr || out == nullptr ||
+      idx_stride < 1)
+    return HGA_ERR_INVALID_ARG;
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.kv = make_kv_view(kv);
+  a.sv = make_sum_view(kv, nullptr, nullptr, nullptr);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  a.C = a.g = a.k = a.G = 1;
+  a.n_pad = 2;
+  a.kcap = 1;
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.out = out;
+  a.lse = lse;
+  a.idx_in = idx;
+  a.n_idx_in = n_idx;
+  a.idx_stride = idx_stride;
+  return run_routed<kModeAttend>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                      const void* group_sum, const hga_params* p, float* out, float* lse,
+                      int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || group_sum == nullptr ||
+      !aligned16(chunk_sum) || !aligned16(group_sum) || out == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
+  if (idx != nullptr && idx_stride < max_routed(kv, p)) return HGA_ERR_INVALID_ARG;
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.kv = make_kv_view(kv);
+  a.sv = make_sum_view(kv, p, chunk_sum, group_sum);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  routing_args(a, kv, p);
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.out = out;
+  a.lse = lse;
+  a.idx_out = idx;
+  a.n_idx_out = n_idx;
+  a.idx_stride = idx ? idx_stride : 0;
+  return run_routed<kModeDecode>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+hga_status hga_set_launch_option(int32_t option, int32_t value) {
+  if (option == HGA_OPT_CTAS_PER_HEAD) {
+    if (value < 0 || value > 16) return HGA_ERR_INVALID_ARG;
+    g_ctas_per_head.store(value);
+    return HGA_OK;
+  }
+  return HGA_ERR_INVALID_ARG;
+}
+
+hga_status hga_get_device_error(cudaStream_t stream, int32_t* bits) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HGA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return HGA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return HGA_ERR_CUDA;
+  }
+  if (bits) *bits = v;
+  if (v & kErrTimeout) return HGA_ERR_TIMEOUT;
+  return v ? HGA_ERR_DEVICE_FAULT : HGA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+/*
+ * hga.h - C ABI of the routed-attention library (libhga.so), sm_100a.
+ *
+ * The method: "Hierarchical Global Attention (HGA)" (Woernle, Fedosov,
+ * Grinenko; arXiv 2606.30709), abstract. A drop-in replacement for dense causal
+ * attention with the pretrained projections unchanged: a query first scores
+ * compact summaries of fixed-size key chunks and keeps the best chunks, then
+ * scores per-group summaries inside them and keeps the best groups, then runs
+ * exact softmax attention over the routed tokens only. The first chunk (sink)
+ * and the last chunk with any partial tail (local) are always kept, following
+ * the keep-beginning-and-end rule of the HISA article ("Hierarchical Indexing
+ * Sparse Attention", shijienb.com summary, two-step block-then-token filter).
+ *
+ * The library takes post-projection, post-rotary q and K (the caller applies the
+ * rotary embedding) plus V, and returns the attention output before the output
+ * projection.
+ *
+ * Conventions shared by every call:
+ *   - All data pointers are DEVICE pointers owned by the caller, except the
+ *     hga_kv / hga_params structs themselves, which are read on the host during
+ *     the call and may be freed on return.
+ *   - bfloat16 tensors are passed as raw 16-bit patterns (`const void*`), 16-byte
+ *     aligned; int32/float tensors are naturally aligned.
+ *   - Calls are asynchronous on `stream`. The library allocates no device
+ *     memory; its only state is one device error word per device (a __device__
+ *     variable) and a process-wide launch option (hga_set_launch_option).
+ *   - Host validation failures return HGA_ERR_INVALID_ARG or
+ *     HGA_ERR_UNSUPPORTED synchronously with nothing enqueued. Problems only the
+ *     device can see (a sequence length above max_len, a page id outside the
+ *     pool, a token index outside its sequence) make the kernel skip the
+ *     offending access and set the device error word, read and cleared by
+ *     hga_get_device_error. No kernel traps.
+ *
+ * Supported sizes: head_dim 64 or 128; n_q_heads % n_kv_heads == 0 with at most
+ * 8 query heads per KV head; chunk % group == 0, chunk / group <= 32;
+ * floor(max_len / chunk) <= 4096; 1 <= top_groups <= chunk / group;
+ * top_chunks >= 1.
+ */
+#ifndef HGA_H_
+#define HGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HGA_OK = 0,
+  HGA_ERR_INVALID_ARG = 1,  /* bad pointer, size or parameter; nothing enqueued */
+  HGA_ERR_UNSUPPORTED = 2,  /* valid but outside the supported sizes above; nothing enqueued */
+  HGA_ERR_CUDA = 3,         /* a CUDA runtime call failed (see cudaGetLastError) */
+  HGA_ERR_DEVICE_FAULT = 4, /* a kernel met a bad device-side input and skipped it */
+  HGA_ERR_TIMEOUT = 5       /* a bounded device wait ran out */
+} hga_status;
+
+/*
+ * Routing parameters. The paper's abstract fixes the two-level order (chunks,
+ * then groups) but not the sizes; these are the caller's choice.
+ */
+typedef struct {
+  int32_t chunk;      /* C: tokens per chunk (one summary per full chunk) */
+  int32_t group;      /* g: tokens per group, chunk % group == 0 */
+  int32_t top_chunks; /* k: routed chunks kept among chunks 1 .. nf-2 */
+  int32_t top_groups; /* G: groups kept in each routed chunk */
+  float scale;        /* softmax scale; 0 means 1/sqrt(head_dim). Routing never scales. */
+} hga_params;
+
+/*
+ * The key/value cache.
+ *   Contiguous (page_table == NULL): k, v are [batch][n_kv_heads][max_len][head_dim].
+ *   Paged: k, v are a page pool [num_pages][n_kv_heads][page_size][head_dim];
+ *   token t of sequence b sits in page page_table[b * max_pages + t / page_size]
+ *   at row t % page_size. Paged caches require page_size == chunk, so one page is
+ *   one chunk and summaries are indexed by physical page.
+ * seq_lens[b] (device) is the number of valid tokens of sequence b, at most max_len.
+ * A decode query of sequence b sits at position seq_lens[b] - 1; its own key and
+ * value are already in the cache.
+ */
+typedef struct {
+  const void* k;
+  const void* v;
+  const int32_t* page_table; /* device, [batch][max_pages], or NULL */
+  const int32_t* seq_lens;   /* device, [batch] */
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t max_len;
+  int32_t page_size; /* paged only */
+  int32_t max_pages; /* paged only: page-table row length, max_pages * page_size >= max_len */
+  int32_t num_pages; /* paged only: pages in the pool */
+} hga_kv;
+
+/*
+ * Summary buffers (bfloat16), written by hga_build_summaries, read by routing.
+ *   Contiguous: chunk_sum [batch][n_kv_heads][max_len/chunk][head_dim]
+ *               group_sum [batch][n_kv_heads][max_len/chunk][chunk/group][head_dim]
+ *   Paged:      chunk_sum [num_pages][n_kv_heads][head_dim]
+ *               group_sum [num_pages][n_kv_heads][chunk/group][head_dim]
+ * hga_summary_bytes reports both sizes.
+ */
+hga_status hga_summary_bytes(const hga_kv* kv, const hga_params* p, size_t* chunk_bytes,
+                             size_t* group_bytes);
+
+/*
+ * Build chunk and group summaries from the post-rotary keys (the abstract's
+ * per-chunk summaries, which see positions through the rotary embedding).
+ * Summary of chunk c: the mean of
+ * K_t over t in [c*C, (c+1)*C); of group j of chunk c: the mean over
+ * [c*C + j*g, c*C + (j+1)*g). fp32 accumulation, bfloat16 round-to-nearest
+ * store. Only full chunks (c < seq_lens[b] / C) are written; other entries are
+ * left untouched. One pass over K; run it after filling the cache.
+ */
+hga_status hga_build_summaries(const hga_kv* kv, const hga_params* p, void* chunk_sum,
+                               void* group_sum, cudaStream_t stream);
+
+/*
+ * Upper bound on the routed tokens of one (sequence, KV head) over every
+ * sequence length up to kv->max_len: the minimum idx_stride for hga_route,
+ * hga_attend and hga_decode. Returns -1 on invalid arguments.
+ */
+int32_t hga_max_routed_tokens(const hga_kv* kv, const hga_params* p);
+
+/*
+ * Two-level routing (abstract: chunks are picked by their summaries first, then
+ * only the best groups inside the picked chunks are kept). Per sequence b and
+ * KV head h, with the R = n_q_heads /
+ * n_kv_heads query heads i of h, nf = seq_lens[b] / chunk full chunks:
+ *   nf <= 2: every token [0, L) is routed.
+ *   else: chunk score sigma_c = sum_i q_i . s_c over candidates c in [1, nf-2];
+ *         keep the top_chunks highest (ties: lower c); inside each kept chunk
+ *         group score tau_{c,j} = sum_i q_i . s_{c,j}, keep the top_groups highest
+ *         (ties: lower j); token list = [0, C) + kept groups (ascending) +
+ *         [(nf-1)*C, L).
+ *   q       [batch][n_q_heads][head_dim] bfloat16, post-rotary
+ *   idx     [batch][n_kv_heads][idx_stride] int32 out: routed positions, ascending
+ *   n_idx   [batch][n_kv_heads] int32 out: number of routed positions
+ * idx_stride must be >= hga_max_routed_tokens(kv, p).
+ */
+hga_status hga_route(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                     const void* group_sum, const hga_params* p, int32_t* idx, int32_t idx_stride,
+                     int32_t* n_idx, cudaStream_t stream);
+
+/*
+ * Exact softmax attention over a given token set (abstract: attention over the
+ * routed tokens is exact, not approximated). For every query head i of KV head h:
+ *   out[b][i] = sum_t softmax_t(scale * q_i . K_t) V_t over t in idx[b][h][0:n_idx]
+ *   lse[b][i] = log sum_t exp(scale * q_i . K_t)    (natural log; lse may be NULL)
+ * The R query heads of a KV head share every K/V tile. An empty set gives
+ * out = 0 and lse = -inf. Tokens must lie in [0, seq_lens[b]); others are skipped
+ * and reported through the device error word.
+ *   out [batch][n_q_heads][head_dim] float32, lse [batch][n_q_heads] float32.
+ * Only p->scale is read from p.
+ */
+hga_status hga_attend(const void* q, int32_t n_q_heads, const hga_kv* kv, const int32_t* idx,
+                      int32_t idx_stride, const int32_t* n_idx, const hga_params* p, float* out,
+                      float* lse, cudaStream_t stream);
+
+/*
+ * Fused decode step: hga_route followed by hga_attend in one kernel, the
+ * routed positions kept on chip. idx / n_idx are optional outputs (both NULL,
+ * or both set with idx_stride >= hga_max_routed_tokens).
+ */
+hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                      const void* group_sum, const hga_params* p, float* out, float* lse,
+                      int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream);
+
+/*
+ * Launch tuning, process-wide (not thread-safe against concurrent calls).
+ *   HGA_OPT_CTAS_PER_HEAD: CTAs (one thread-block cluster) that cooperate on one
+ *   (sequence, KV head) in hga_route / hga_attend / hga_decode; 0 = automatic,
+ *   1..16 otherwise (above 8 needs non-portable cluster support).
+ * Returns HGA_ERR_INVALID_ARG for an unknown option or value.
+ */
+enum { HGA_OPT_CTAS_PER_HEAD = 1 };
+hga_status hga_set_launch_option(int32_t option, int32_t value);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word.
+ * HGA_OK if no kernel reported a problem since the last call,
+ * HGA_ERR_DEVICE_FAULT for a bad device-side input, HGA_ERR_TIMEOUT for an
+ * expired bounded wait, HGA_ERR_CUDA if the synchronisation itself failed.
+ * `bits` (may be NULL) receives the raw word: 1 sequence length, 2 page id,
+ * 4 token index, 8 timeout.
+ */
+hga_status hga_get_device_error(cudaStream_t stream, int32_t* bits);
+
+/* Static description of a status code. */
+const char* hga_status_string(hga_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H_ */

@@ -1,0 +1,123 @@
+"""C ABI checks that need no GPU: the library loads, exports every call that
+include/hga.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import hierarchical_routed_sparse_build_b200 as hga
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hga.h")
+
+INVALID, UNSUPPORTED = 1, 2
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any launch
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hga_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_all_exported():
+    names = declared_functions()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(hga.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(hga.EXPORTED)
+
+
+def test_status_strings():
+    for s in range(6):
+        assert hga.hga_status_string(s)
+    assert hga.hga_status_string(99) == "unknown status"
+
+
+def kv_desc(**over):
+    d = dict(k=FAKE, v=FAKE, seq_lens=FAKE, n_kv_heads=4, head_dim=128, max_len=65536, batch=2)
+    d.update(over)
+    return hga.make_kv(d.pop("k"), d.pop("v"), d.pop("seq_lens"), **d)
+
+
+def params(**over):
+    d = dict(chunk=128, group=16, top_chunks=32, top_groups=4, scale=0.0)
+    d.update(over)
+    return hga.make_params(**d)
+
+
+def raw_decode(kv, p, q=FAKE, hq=32, out=FAKE, idx=None, stride=0, n_idx=None):
+    return hga._lib.hga_decode(q, hq, ctypes.byref(kv), FAKE, FAKE, ctypes.byref(p), out, None, idx, stride,
+                               n_idx, None)
+
+
+@pytest.mark.parametrize("kv_over,p_over,hq,want", [
+    (dict(k=0), {}, 32, INVALID),                      # null K
+    (dict(seq_lens=0), {}, 32, INVALID),               # null lengths
+    (dict(head_dim=96), {}, 32, UNSUPPORTED),          # head dim
+    (dict(batch=0), {}, 32, INVALID),
+    (dict(k=FAKE + 8), {}, 32, INVALID),               # misaligned
+    ({}, dict(group=24), 32, INVALID),                 # g does not divide C
+    ({}, dict(top_groups=9), 32, INVALID),             # G > C/g
+    ({}, dict(top_chunks=0), 32, INVALID),
+    ({}, dict(chunk=256, group=4), 32, UNSUPPORTED),   # C/g > 32
+    ({}, dict(scale=-1.0), 32, INVALID),
+    ({}, {}, 30, INVALID),                             # Hq % Hkv != 0
+    ({}, {}, 48, UNSUPPORTED),                         # 12 query heads per KV head
+    (dict(max_len=4096 * 128 + 128), {}, 32, UNSUPPORTED),  # more than 4096 chunks
+    (dict(page_table=FAKE, page_size=64, max_pages=1024, num_pages=8), {}, 32, UNSUPPORTED),  # page != chunk
+    (dict(page_table=FAKE, page_size=128, max_pages=4, num_pages=8), {}, 32, INVALID),  # table too short
+])
+def test_decode_rejects_bad_arguments_on_host(kv_over, p_over, hq, want):
+    assert raw_decode(kv_desc(**kv_over), params(**p_over), hq=hq) == want
+
+
+def test_decode_output_and_index_arguments():
+    kv, p = kv_desc(), params()
+    assert raw_decode(kv, p, out=0) == INVALID
+    assert raw_decode(kv, p, q=0) == INVALID
+    assert raw_decode(kv, p, idx=FAKE, stride=4096, n_idx=None) == INVALID  # idx without n_idx
+    assert raw_decode(kv, p, idx=FAKE, stride=100, n_idx=FAKE) == INVALID   # stride below the bound
+
+
+def test_route_and_attend_validation():
+    kv, p = kv_desc(), params()
+    L = hga._lib
+    assert L.hga_route(FAKE, 32, ctypes.byref(kv), FAKE, FAKE, ctypes.byref(p), FAKE, 10, FAKE, None) == INVALID
+    assert L.hga_route(FAKE, 32, ctypes.byref(kv), None, FAKE, ctypes.byref(p), FAKE, 4096, FAKE, None) == INVALID
+    assert L.hga_attend(FAKE, 32, ctypes.byref(kv), None, 16, FAKE, ctypes.byref(p), FAKE, None, None) == INVALID
+    assert L.hga_attend(FAKE, 32, ctypes.byref(kv_desc(v=0)), FAKE, 16, FAKE, ctypes.byref(p), FAKE, None,
+                        None) == INVALID
+    assert L.hga_build_summaries(ctypes.byref(kv), ctypes.byref(p), None, FAKE, None) == INVALID
+    assert L.hga_build_summaries(None, ctypes.byref(p), FAKE, FAKE, None) == INVALID
+
+
+@pytest.mark.parametrize("max_len,C,g,k,G", [
+    (65536, 128, 16, 32, 4), (16384, 128, 16, 16, 4), (4096, 64, 16, 8, 2), (100, 64, 16, 8, 2),
+    (65536 + 77, 128, 16, 32, 4), (1000, 16, 4, 100, 4), (383, 128, 16, 2, 1), (384, 128, 16, 2, 1),
+])
+def test_max_routed_tokens_bounds_every_length(max_len, C, g, k, G):
+    kv = kv_desc(max_len=max_len, head_dim=64)
+    n = hga.hga_max_routed_tokens(kv, params(chunk=C, group=g, top_chunks=k, top_groups=G))
+    want = max(oracle.max_routed(L, C, g, k, G) for L in range(1, max_len + 1))
+    assert n == want
+
+
+def test_summary_bytes():
+    kv = kv_desc()
+    cb, gb = hga.hga_summary_bytes(kv, params())
+    assert cb == 2 * 4 * 512 * 128 * 2 and gb == cb * 8
+    kvp = kv_desc(page_table=FAKE, page_size=128, max_pages=512, num_pages=1000)
+    cb, gb = hga.hga_summary_bytes(kvp, params())
+    assert cb == 1000 * 4 * 128 * 2 and gb == cb * 8
+
+
+def test_launch_option_validation():
+    with pytest.raises(hga.HgaError):
+        hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 17)
+    with pytest.raises(hga.HgaError):
+        hga.hga_set_launch_option(7, 1)
+    hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
