@@ -7,12 +7,12 @@
  * does, and it shares no code with the CUDA kernels.
  *
  * Source of the method: "Hierarchical Global Attention (HGA)" (Woernle,
- * Fedosov, Grinenko; arXiv 2606.30709), abstract: routing first retrieves
- * relevant chunks with compact RoPE-aware summaries, then keeps only the most
- * relevant groups inside them, then performs exact token-level attention over
- * the retrieved set. The rule that the beginning and the end of the text are
- * always kept comes from the HISA article ("Hierarchical Indexing Sparse
- * Attention", shijienb.com summary, two-step block-then-token filter).
+ * Fedosov, Grinenko; arXiv 2606.30709), abstract: a query scores per-chunk
+ * summaries of the rotary-embedded keys and keeps the best chunks, narrows to
+ * the best groups inside those chunks, and attends exactly to the tokens of the
+ * kept groups. Keeping the start and the end of the context in every selection
+ * follows the HISA article ("Hierarchical Indexing Sparse Attention",
+ * shijienb.com summary, two-step block-then-token filter).
  *
  * Readings taken where the pages leave a step open (each is listed with its
  * reason in the design notes):
