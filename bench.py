@@ -191,7 +191,7 @@ def run_gpu(args, rank: int, world: int, dist):
     st, bits = hga.hga_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error after setup: {bits}")
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
         cache.decode(q, out, lse)
@@ -201,7 +201,7 @@ def run_gpu(args, rank: int, world: int, dist):
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         for i in range(n):
             if per_step_flush:
-                flush.zero_()
+                flush.max()
             starts[i].record(stream)
             fn()
             ends[i].record(stream)
@@ -294,7 +294,7 @@ def run_gpu(args, rank: int, world: int, dist):
                                "local, top-4 groups (2304 routed tokens per KV head, 3.5%)",
                    "batch_per_gpu": B, "ctx_len": w.ctx_len, "distinct_sequences": min(B, args.distinct),
                    "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
-                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "l2": "flushed between steps (256 MiB read, outside the timed events)",
                    "ctas_per_head": args.ctas or "auto"},
         "roofline": {"bound": "hbm", "kernel": "routed_kernel<128, decode> (whole step, one launch)",
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",

@@ -88,8 +88,9 @@ int sm_count() {
 int pick_cluster(int units) {
   int P = g_ctas_per_head.load();
   if (P > 0) return P;
-  // about two co-resident CTAs per SM in total, at most 8 per (sequence, KV head)
-  P = (2 * sm_count() + units - 1) / units;
+  // as many CTAs per (sequence, KV head) as fit in one wave of two CTAs per SM,
+  // at most 8 (the portable cluster size)
+  P = (2 * sm_count()) / units;
   return P < 1 ? 1 : (P > 8 ? 8 : P);
 }
 
@@ -123,16 +124,38 @@ float scale_log2(const hga_params* p, int d) {
   return (float)(sc * 1.4426950408889634074);
 }
 
+// Kernel attributes are set once per (kernel, device) and raised only when a
+// launch needs more, keeping the per-call host cost to the launch itself.
+constexpr int kMaxDevices = 64;
+
 template <int D, int MODE>
-cudaError_t launch_routed(const RoutedArgs& a, int units, int P, cudaStream_t stream) {
-  const RoutedSmem lay(D, a.n_pad, a.kcap, a.G);
-  auto kern = routed_kernel<D, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+cudaError_t configure_routed(int smem_bytes, bool non_portable) {
+  static std::atomic<int> smem_set[kMaxDevices];
+  static std::atomic<bool> np_set[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (P > 8) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  auto kern = routed_kernel<D, MODE>;
+  if (smem_bytes > smem_set[dev].load()) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess) return e;
+    smem_set[dev].store(smem_bytes);
+  }
+  if (non_portable && !np_set[dev].load()) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    np_set[dev].store(true);
   }
+  return cudaSuccess;
+}
+
+template <int D, int MODE>
+cudaError_t launch_routed(const RoutedArgs& a, int units, int P, cudaStream_t stream) {
+  const RoutedSmem lay(D, a.n_pad, a.kcap, a.G, a.C / a.g);
+  auto kern = routed_kernel<D, MODE>;
+  cudaError_t e = configure_routed<D, MODE>(lay.total, P > 8);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3((unsigned)(units * P), 1, 1);
@@ -149,8 +172,11 @@ cudaError_t launch_routed(const RoutedArgs& a, int units, int P, cudaStream_t st
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+constexpr int kMaxSmemPerCta = 227 * 1024;
+
 template <int MODE>
 hga_status run_routed(RoutedArgs a, int D, int units, cudaStream_t stream) {
+  if (RoutedSmem(D, a.n_pad, a.kcap, a.G, a.C / a.g).total > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
   const int P = pick_cluster(units);
   cudaError_t e = D == 128 ? launch_routed<128, MODE>(a, units, P, stream)
                            : launch_routed<64, MODE>(a, units, P, stream);

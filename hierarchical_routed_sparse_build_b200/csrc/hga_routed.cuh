@@ -10,14 +10,15 @@
 // The P CTAs of a cluster split every phase and meet at hardware cluster
 // barriers; partial results move through distributed shared memory (DSMEM),
 // so nothing goes through global scratch memory:
-//   R1  chunk scores: each CTA scores 1/P of the candidate chunks 1..nf-2 with
-//       the head-summed query (sum_i q_i . s_c = (sum_i q_i) . s_c) and writes
-//       the 64-bit keys (score, then lower id) into every CTA's shared memory.
+//   R1  chunk scores: each CTA stages 1/P of the candidate chunk summaries
+//       (chunks 1..nf-2) with coalesced cp.async, scores them thread-per-row
+//       against the head-summed query (sum_i q_i . s_c = (sum_i q_i) . s_c) and
+//       writes the 64-bit keys (score bits, then lower id) into every CTA.
 //   --  cluster barrier
-//   R2  every CTA sorts all keys (bitonic, shared memory) and takes the top k;
-//       kept chunk ids are put in ascending order.
-//   R3  group scores: each CTA scores the groups of 1/P of the kept chunks and
-//       broadcasts a bit mask of the top-G groups per chunk.
+//   R2  every CTA finds the k-th largest key of all candidates (bucket select)
+//       and keeps the keys at or above it, in ascending chunk order.
+//   R3  group scores: each CTA stages and scores the groups of 1/P of the kept
+//       chunks and broadcasts a bit mask of the top-G groups per chunk.
 //   --  cluster barrier
 //   A   attention: the routed list (sink, kept groups, local) is cut into
 //       16-token tiles; each CTA takes 1/P of them, its warps take tiles
@@ -40,8 +41,13 @@ namespace cg = cooperative_groups;
 
 enum RoutedMode : int { kModeRoute = 1, kModeAttend = 2, kModeDecode = 3 };
 
-constexpr int kRoutedWarps = 4;
+constexpr int kRoutedWarps = 6;
 constexpr int kRoutedThreads = kRoutedWarps * 32;
+constexpr int kBuckets = 1024;             // bucket-select histogram size
+// misc[] (32 ints): [0..5] select state, [8..15] per-warp min, [16..23] per-warp
+// max, [24..31] per-warp scan totals
+static_assert(kRoutedWarps <= 8, "misc[] holds at most 8 per-warp slots");
+constexpr int kStageBytes = 32 * 1024;     // routing: double-buffered summary staging
 
 struct RoutedArgs {
   KvView kv;
@@ -49,7 +55,7 @@ struct RoutedArgs {
   const uint16_t* q;  // [B][Hq][D]
   int hq, R;
   int C, g, k, G;     // routing parameters (G already <= C/g)
-  int n_pad;          // power of two >= max candidates (max_chunks - 2), >= 2
+  int n_pad;          // >= max candidates (max_chunks - 2), >= 2
   int kcap;           // >= kept chunks for any length (min(k, max_chunks - 2)), >= 1
   float scale_log2;   // softmax scale * log2(e)
   float* out;         // [B][Hq][D]
@@ -61,72 +67,236 @@ struct RoutedArgs {
   int idx_stride;
 };
 
-// Shared-memory carve-up (byte offsets), identical on host and device.
+// Shared-memory carve-up (byte offsets), identical on host and device. One
+// union region serves, in turn, the routing keys plus the summary staging
+// area, the per-warp attention tiles, and the per-warp partial outputs.
 struct RoutedSmem {
-  int qsum, keys, sel_tmp, sel, gmask, gstart, gsc, rows, red_o, red_m, red_l, cta_o, cta_m, cta_l,
-      qfrag, total;
+  int qsum, sel, gmask, gstart, rows, red_m, red_l, cta_o, cta_m, cta_l, qfrag, hist, misc, gsc,
+      uni, keys, stage, stage_rows, tiles, red_o, total;
   __host__ __device__ static int up16(int x) { return (x + 15) & ~15; }
-  __host__ __device__ RoutedSmem(int D, int n_pad, int kcap, int gk) {
+  __host__ __device__ RoutedSmem(int D, int n_pad, int kcap, int gk, int gpc) {
     int o = 0;
     qsum = o;    o = up16(o + 4 * D);
-    keys = o;    o = up16(o + 8 * n_pad);
-    sel_tmp = o; o = up16(o + 4 * kcap);
     sel = o;     o = up16(o + 4 * kcap);
     gmask = o;   o = up16(o + 4 * kcap);
     gstart = o;  o = up16(o + 4 * kcap * gk);
-    gsc = o;     o = up16(o + 4 * kRoutedWarps * 32);
     rows = o;    o = up16(o + 4 * kEntryBatch);
-    red_o = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv * D);
     red_m = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
     red_l = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
     cta_o = o;   o = up16(o + 4 * kMaxHeadsPerKv * D);
     cta_m = o;   o = up16(o + 4 * kMaxHeadsPerKv);
     cta_l = o;   o = up16(o + 4 * kMaxHeadsPerKv);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
+    hist = o;    o = up16(o + 4 * kBuckets);
+    misc = o;    o = up16(o + 4 * 32);
+    // union: {keys, staging} during routing | per-warp tiles | partial outputs
+    uni = o;
+    keys = o;
+    stage = up16(keys + 8 * n_pad);
+    stage_rows = kStageBytes / (2 * D);
+    tiles = o;
+    red_o = o;
+    int u = stage + kStageBytes - o;
+    const int tiles_bytes = kRoutedWarps * 16 * D * 2;
+    const int red_bytes = 4 * kRoutedWarps * kMaxHeadsPerKv * D;
+    if (tiles_bytes > u) u = tiles_bytes;
+    if (red_bytes > u) u = red_bytes;
+    o = up16(o + u);
+    gsc = o;     o = up16(o + 4 * kcap * gpc);
     total = o;
   }
 };
 
-// Block-wide bitonic sort of n (power of two) keys, descending.
-__device__ __forceinline__ void bitonic_sort_desc(uint64_t* keys, int n) {
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t a = keys[lo], b = keys[hi];
-        if ((a < b) == desc) {
-          keys[lo] = b;
-          keys[hi] = a;
+// Block-wide exclusive prefix sum of one int per thread (kRoutedThreads).
+__device__ __forceinline__ int block_exclusive_scan(int x, int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+  __syncthreads();
+  return before + incl - x;
+}
+
+// Staged summary rows: unit u of staged row i sits at slot i*U + (u ^ (i % U)),
+// so row-wise stores and thread-per-row reads are both bank-conflict-free.
+template <int D>
+__device__ __forceinline__ int stage_slot(int i, int u) {
+  return i * (D / 8) + (u ^ (i & (D / 8 - 1)));
+}
+
+// Head-summed score of staged row i: qsum . row (fp32).
+template <int D>
+__device__ __forceinline__ float staged_row_dot(const uint4* stage, int i, const float* qsum) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int u = 0; u < D / 8; ++u) {
+    const uint4 v = stage[stage_slot<D>(i, u)];
+    const float4 a = *reinterpret_cast<const float4*>(qsum + 8 * u);
+    const float4 c = *reinterpret_cast<const float4*>(qsum + 8 * u + 4);
+    s0 = fmaf(bf16_lo(v.x), a.x, s0);
+    s1 = fmaf(bf16_hi(v.x), a.y, s1);
+    s0 = fmaf(bf16_lo(v.y), a.z, s0);
+    s1 = fmaf(bf16_hi(v.y), a.w, s1);
+    s0 = fmaf(bf16_lo(v.z), c.x, s0);
+    s1 = fmaf(bf16_hi(v.z), c.y, s1);
+    s0 = fmaf(bf16_lo(v.w), c.z, s0);
+    s1 = fmaf(bf16_hi(v.w), c.w, s1);
+  }
+  return s0 + s1;
+}
+
+// Stream n_rows summary rows through the staging area in two alternating
+// buffers (cp.async groups), so the copies of block i+1 are in flight while
+// block i is scored. src(row) gives the global address of a row; consume(buf,
+// first_row, n) scores rows first_row .. first_row+n-1 staged at buf
+// (stage_slot layout, local row index). Every thread of the CTA must call it.
+template <int D, typename Src, typename Consume>
+__device__ __forceinline__ void stream_rows(uint4* stage, int stage_rows, int n_rows, Src src,
+                                            Consume consume) {
+  constexpr int U = D / 8;
+  const int half = stage_rows / 2;
+  auto issue = [&](int first, uint4* buf) {
+    const int n = min(half, n_rows - first);
+    for (int p = threadIdx.x; p < n * U; p += kRoutedThreads) {
+      const int i = p / U, u = p - i * U;
+      cp_async16(buf + stage_slot<D>(i, u), src(first + i) + 8 * u);
+    }
+  };
+  uint4* bufs[2] = {stage, stage + half * U};
+  if (0 < n_rows) issue(0, bufs[0]);
+  cp_async_commit();
+  if (half < n_rows) issue(half, bufs[1]);
+  cp_async_commit();
+  int which = 0;
+  for (int first = 0; first < n_rows; first += half) {
+    cp_async_wait<1>();
+    __syncthreads();
+    consume(bufs[which], first, min(half, n_rows - first));
+    __syncthreads();
+    if (first + 2 * half < n_rows) issue(first + 2 * half, bufs[which]);
+    cp_async_commit();
+    which ^= 1;
+  }
+  cp_async_wait<0>();
+}
+
+// Top-r selection over n unique keys; keys[i] belongs to candidate chunk i+1
+// (key = order-preserving score bits << 32 | ~id, so larger key = higher score,
+// then lower id: the oracle's order). Finds the r-th largest key K_r exactly and
+// writes the ids of all keys >= K_r, ascending, to sel[0..r):
+//   1. bucket the 32-bit score parts linearly between their block min and max
+//      (a monotone map), histogram, and find the bucket b* holding the r-th;
+//   2. compact the keys of b* and rank them exactly (64-bit compare) to get K_r;
+//   3. ordered compaction of keys >= K_r (candidate order = ascending ids).
+// scratch must hold scratch_cap keys; if b* holds more, ranking falls back to
+// scanning all n keys (correct, slower; only for near-constant scores).
+__device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, int r, int* sel,
+                                                  int* hist, int* misc, uint64_t* scratch,
+                                                  int scratch_cap) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = tid; i < n; i += kRoutedThreads) {
+    const uint32_t u = (uint32_t)(keys[i] >> 32);
+    lo = min(lo, u);
+    hi = max(hi, u);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, off));
+    hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, off));
+  }
+  if (lane == 0) {
+    misc[8 + warp] = (int)lo;
+    misc[16 + warp] = (int)hi;
+  }
+  for (int i = tid; i < kBuckets; i += kRoutedThreads) hist[i] = 0;
+  if (tid == 0) misc[2] = 0;
+  __syncthreads();
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
+#pragma unroll
+  for (int w = 0; w < kRoutedWarps; ++w) {
+    lo = min(lo, (uint32_t)misc[8 + w]);
+    hi = max(hi, (uint32_t)misc[16 + w]);
+  }
+  const float scale = (float)kBuckets / ((float)(hi - lo) + 1.0f);
+  auto bucket = [&](uint32_t u) { return min(kBuckets - 1, (int)((float)(u - lo) * scale)); };
+  for (int i = tid; i < n; i += kRoutedThreads) atomicAdd(&hist[bucket((uint32_t)(keys[i] >> 32))], 1);
+  __syncthreads();
+  if (warp == 0) {
+    constexpr int PER = kBuckets / 32;
+    int tot = 0;
+    for (int k = 0; k < PER; ++k) tot += hist[kBuckets - 1 - PER * lane - k];
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const int excl = incl - tot;
+    if (excl < r && r <= incl) {
+      int acc = excl;
+      for (int k = 0; k < PER; ++k) {
+        const int b = kBuckets - 1 - PER * lane - k;
+        if (acc + hist[b] >= r) {
+          misc[0] = b;
+          misc[1] = acc;
+          break;
         }
+        acc += hist[b];
       }
-      __syncthreads();
     }
   }
-}
-
-// Dot product of one bf16 summary row (16 B per lane, LPR lanes) with qsum.
-template <int D>
-__device__ __forceinline__ float row_dot_partial(const uint4& v, const float* qsum, int col) {
-  const float4 a = *reinterpret_cast<const float4*>(qsum + col);
-  const float4 c = *reinterpret_cast<const float4*>(qsum + col + 4);
-  float s = bf16_lo(v.x) * a.x;
-  s = fmaf(bf16_hi(v.x), a.y, s);
-  s = fmaf(bf16_lo(v.y), a.z, s);
-  s = fmaf(bf16_hi(v.y), a.w, s);
-  s = fmaf(bf16_lo(v.z), c.x, s);
-  s = fmaf(bf16_hi(v.z), c.y, s);
-  s = fmaf(bf16_lo(v.w), c.z, s);
-  s = fmaf(bf16_hi(v.w), c.w, s);
-  return s;
-}
-
-template <int LPR>
-__device__ __forceinline__ float reduce_lanes(float s) {
-#pragma unroll
-  for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
-  return s;
+  __syncthreads();
+  const int bstar = misc[0], need = r - misc[1];
+  const int members = hist[bstar];
+  const bool in_scratch = members <= scratch_cap;
+  if (in_scratch) {
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const uint64_t key = keys[i];
+      if (bucket((uint32_t)(key >> 32)) == bstar) scratch[atomicAdd(&misc[2], 1)] = key;
+    }
+    __syncthreads();
+    for (int m = tid; m < members; m += kRoutedThreads) {
+      const uint64_t km = scratch[m];
+      int rank = 0;
+      for (int j = 0; j < members; ++j) rank += scratch[j] > km;
+      if (rank == need - 1) {
+        misc[4] = (int)(uint32_t)(km >> 32);
+        misc[5] = (int)(uint32_t)(km & 0xFFFFFFFFu);
+      }
+    }
+  } else {
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const uint64_t km = keys[i];
+      if (bucket((uint32_t)(km >> 32)) != bstar) continue;
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint64_t kj = keys[j];
+        rank += (kj > km) && bucket((uint32_t)(kj >> 32)) == bstar;
+      }
+      if (rank == need - 1) {
+        misc[4] = (int)(uint32_t)(km >> 32);
+        misc[5] = (int)(uint32_t)(km & 0xFFFFFFFFu);
+      }
+    }
+  }
+  __syncthreads();
+  const uint64_t kth = ((uint64_t)(uint32_t)misc[4] << 32) | (uint64_t)(uint32_t)misc[5];
+  const int per = (n + kRoutedThreads - 1) / kRoutedThreads;
+  const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
+  int cnt = 0;
+  for (int i = s0; i < s1; ++i) cnt += keys[i] >= kth;
+  int pos = block_exclusive_scan(cnt, misc + 24);
+  for (int i = s0; i < s1; ++i)
+    if (keys[i] >= kth) sel[pos++] = (int)route_key_id(keys[i]);
 }
 
 template <int D, int MODE>
@@ -142,17 +312,19 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr bool kRouting = (MODE & kModeRoute) != 0;
   constexpr bool kAttention = (MODE & kModeAttend) != 0;
-  constexpr int LPR = D / 8, RPI = 32 / LPR;
 
   const int gk = a.G;
-  const RoutedSmem lay(D, a.n_pad, a.kcap, gk);
+  const RoutedSmem lay(D, a.n_pad, a.kcap, gk, a.C / a.g);
   float* qsum = reinterpret_cast<float*>(smem + lay.qsum);
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem + lay.keys);
-  int* sel_tmp = reinterpret_cast<int*>(smem + lay.sel_tmp);
+  uint4* stage = reinterpret_cast<uint4*>(smem + lay.stage);
+  const int stage_rows = lay.stage_rows;
+  int* hist = reinterpret_cast<int*>(smem + lay.hist);
+  int* misc = reinterpret_cast<int*>(smem + lay.misc);
+  float* gsc = reinterpret_cast<float*>(smem + lay.gsc);
   int* sel = reinterpret_cast<int*>(smem + lay.sel);
   uint32_t* gmask = reinterpret_cast<uint32_t*>(smem + lay.gmask);
   int* gstart = reinterpret_cast<int*>(smem + lay.gstart);
-  float* gsc = reinterpret_cast<float*>(smem + lay.gsc);
   uint32_t* rows = reinterpret_cast<uint32_t*>(smem + lay.rows);
   float* red_o = reinterpret_cast<float*>(smem + lay.red_o);
   float* red_m = reinterpret_cast<float*>(smem + lay.red_m);
@@ -161,6 +333,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
   float* cta_m = reinterpret_cast<float*>(smem + lay.cta_m);
   float* cta_l = reinterpret_cast<float*>(smem + lay.cta_l);
   uint4* qfrag = reinterpret_cast<uint4*>(smem + lay.qfrag);
+  uint4* tile = reinterpret_cast<uint4*>(smem + lay.tiles) + warp * TileGeom<D>::kTileSlots;
 
   const bool paged = a.kv.page_table != nullptr;
   const int L = a.kv.length(b);
@@ -174,6 +347,17 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
   const int r = n_cand < a.k ? n_cand : a.k;
   int S = 0;  // routed entries
 
+  // physical page of chunk c (paged caches; 0 after reporting a bad entry)
+  auto chunk_page = [&](int c) -> int {
+    if (!paged) return 0;
+    const int page = __ldg(a.kv.page_table + (int64_t)b * a.kv.max_pages + c);
+    if ((unsigned)page >= (unsigned)a.kv.num_pages) {
+      report_error(kErrPage);
+      return 0;  // read a real row; results after a reported error are unspecified
+    }
+    return page;
+  };
+
   if (kRouting) {
     // Peers write into this CTA's shared memory in R1; every CTA of the cluster
     // must have started first. Arrive now, wait just before the first remote store.
@@ -183,60 +367,33 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
       for (int i = 0; i < a.R; ++i) s += bf16_to_f(qb[(int64_t)i * D + e]);
       qsum[e] = s;
     }
-    for (int i = n_cand + tid; i < a.n_pad; i += kRoutedThreads) keys[i] = 0ull;
     __syncthreads();
-
     cluster_wait();
 
     // R1: score this CTA's share of the candidates; broadcast keys to the cluster.
-    const bool sort_needed = n_cand > r;
-    if (sort_needed) {
+    const bool select_needed = n_cand > r;
+    if (select_needed) {
       const int c0 = (int)((int64_t)n_cand * cr / P), c1 = (int)((int64_t)n_cand * (cr + 1) / P);
-      const int nsg = kRoutedWarps * RPI;
-      const int sg = warp * RPI + lane / LPR;
-      const int col = (lane % LPR) * 8;
-      for (int base = c0; base < c1; base += 4 * nsg) {
-        uint4 v[4];
-        int cand[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          cand[u] = base + sg + u * nsg;
-          v[u] = make_uint4(0, 0, 0, 0);
-          if (cand[u] < c1) {
-            const int c = cand[u] + 1;
-            int page = 0;
-            bool ok = true;
-            if (paged) {
-              page = __ldg(a.kv.page_table + (int64_t)b * a.kv.max_pages + c);
-              ok = (unsigned)page < (unsigned)a.kv.num_pages;
-              if (!ok && (lane % LPR) == 0) report_error(kErrPage);
+      stream_rows<D>(
+          stage, stage_rows, c1 - c0,
+          [&](int i) {
+            const int c = c0 + i + 1;
+            return a.sv.chunk + a.sv.chunk_off(paged, b, h, hkv, c, chunk_page(c));
+          },
+          [&](const uint4* buf, int first, int n) {
+            for (int i = tid; i < n; i += kRoutedThreads) {
+              const int cand = c0 + first + i;
+              const uint64_t key = route_key(staged_row_dot<D>(buf, i, qsum), (uint32_t)(cand + 1));
+              for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(keys, pr)[cand] = key;
             }
-            if (ok) v[u] = ldg_nc(a.sv.chunk + a.sv.chunk_off(paged, b, h, hkv, c, page) + col);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float s = reduce_lanes<LPR>(row_dot_partial<D>(v[u], qsum, col));
-          if (cand[u] < c1 && (lane % LPR) == 0) {
-            const uint64_t key = route_key(s, (uint32_t)(cand[u] + 1));
-            for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(keys, pr)[cand[u]] = key;
-          }
-        }
-      }
+          });
     }
     cluster.sync();
 
-    // R2: top-r chunks, ascending ids.
-    if (sort_needed) {
-      bitonic_sort_desc(keys, a.n_pad);
-      for (int i = tid; i < r; i += kRoutedThreads) sel_tmp[i] = (int)route_key_id(keys[i]);
-      __syncthreads();
-      for (int i = tid; i < r; i += kRoutedThreads) {
-        const int c = sel_tmp[i];
-        int rank = 0;
-        for (int j = 0; j < r; ++j) rank += sel_tmp[j] < c;
-        sel[rank] = c;
-      }
+    // R2: top-r chunks, ascending ids (every CTA, from the full key set).
+    if (select_needed) {
+      select_top_chunks(keys, n_cand, r, sel, hist, misc, reinterpret_cast<uint64_t*>(stage),
+                        (stage_rows * 2 * D) / 8);
     } else {
       for (int i = tid; i < r; i += kRoutedThreads) sel[i] = i + 1;
     }
@@ -246,45 +403,35 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
     const bool all_groups = gk >= gpc;
     if (!all_groups) {
       const int s0 = (int)((int64_t)r * cr / P), s1 = (int)((int64_t)r * (cr + 1) / P);
-      const int sub = lane / LPR, col = (lane % LPR) * 8;
-      for (int i = s0 + warp; i < s1; i += kRoutedWarps) {
-        const int c = sel[i];
-        int page = 0;
-        bool ok = true;
-        if (paged) {
-          page = __ldg(a.kv.page_table + (int64_t)b * a.kv.max_pages + c);
-          ok = (unsigned)page < (unsigned)a.kv.num_pages;
+      const int n_rows = (s1 - s0) * gpc;
+      for (int i = tid; i < s1 - s0; i += kRoutedThreads) gmask[s0 + i] = 0u;
+      stream_rows<D>(
+          stage, stage_rows, n_rows,
+          [&](int i) {
+            const int ci = i / gpc, j = i - ci * gpc;
+            const int c = sel[s0 + ci];
+            return a.sv.group + a.sv.group_off(paged, b, h, hkv, c, chunk_page(c)) + (int64_t)j * D;
+          },
+          [&](const uint4* buf, int first, int n) {
+            for (int i = tid; i < n; i += kRoutedThreads) gsc[first + i] = staged_row_dot<D>(buf, i, qsum);
+          });
+      __syncthreads();
+      for (int i = tid; i < n_rows; i += kRoutedThreads) {
+        const int ci = i / gpc, j = i - ci * gpc;
+        const float tj = gsc[i];
+        const float* row_scores = gsc + ci * gpc;
+        int rank = 0;
+        for (int l = 0; l < gpc; ++l) {
+          const float tl = row_scores[l];
+          rank += (tl > tj) || (tl == tj && l < j);
         }
-        const uint16_t* gbase = a.sv.group + a.sv.group_off(paged, b, h, hkv, c, page) + col;
-        for (int j0 = 0; j0 < gpc; j0 += 4 * RPI) {
-          uint4 v[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = j0 + sub + u * RPI;
-            v[u] = (ok && j < gpc) ? ldg_nc(gbase + (int64_t)j * D) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = j0 + sub + u * RPI;
-            const float s = reduce_lanes<LPR>(row_dot_partial<D>(v[u], qsum, col));
-            if (j < gpc && (lane % LPR) == 0) gsc[warp * 32 + j] = s;
-          }
-        }
-        __syncwarp();
-        bool keep = false;
-        if (lane < gpc) {
-          const float tj = gsc[warp * 32 + lane];
-          int rank = 0;
-          for (int l = 0; l < gpc; ++l) {
-            const float tl = gsc[warp * 32 + l];
-            rank += (tl > tj) || (tl == tj && l < lane);
-          }
-          keep = rank < gk;
-        }
-        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, keep);
-        if (lane == 0)
-          for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(gmask, pr)[i] = mask;
-        __syncwarp();
+        if (rank < gk) atomicOr(&gmask[s0 + ci], 1u << j);
+      }
+      __syncthreads();
+      for (int ci = tid; ci < s1 - s0; ci += kRoutedThreads) {
+        const uint32_t m = gmask[s0 + ci];
+        for (int pr = 0; pr < P; ++pr)
+          if (pr != cr) cluster.map_shared_rank(gmask, pr)[s0 + ci] = m;
       }
     }
     cluster.sync();
@@ -378,8 +525,9 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
       for (int i = tid; i < n_t * 16; i += kRoutedThreads)
         if (rows[i] == kInvalidRow) rows[i] = fallback_row;
       __syncthreads();
-      attend_tiles<D>(st, rows, n_e, warp, kRoutedWarps, Kp, Vp, qfrag, a.scale_log2, lane);
+      attend_tiles<D>(st, rows, n_e, warp, kRoutedWarps, Kp, Vp, qfrag, tile, a.scale_log2, lane);
     }
+    __syncthreads();  // every warp is done with its tile before red_o reuses the region
 
     // warp partials -> shared memory
 #pragma unroll
@@ -407,39 +555,47 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
       }
     }
     __syncthreads();
-    // CTA combine over warps
+    // CTA combine over warps; a single-CTA cluster writes the output directly.
     for (int i = tid; i < a.R * D; i += kRoutedThreads) {
       const int n = i / D, dd = i - n * D;
       float M = -INFINITY;
+#pragma unroll
       for (int w = 0; w < kRoutedWarps; ++w) M = fmaxf(M, red_m[w * kMaxHeadsPerKv + n]);
       float acc = 0.f, den = 0.f;
       if (M != -INFINITY) {
+#pragma unroll
         for (int w = 0; w < kRoutedWarps; ++w) {
-          const float mw = red_m[w * kMaxHeadsPerKv + n];
-          if (mw == -INFINITY) continue;
-          const float f = ex2(mw - M);
+          const float f = ex2(red_m[w * kMaxHeadsPerKv + n] - M);  // -inf -> 0
           acc = fmaf(red_o[(w * kMaxHeadsPerKv + n) * D + dd], f, acc);
           den = fmaf(red_l[w * kMaxHeadsPerKv + n], f, den);
         }
       }
-      cta_o[n * D + dd] = acc;
-      if (dd == 0) {
-        cta_m[n] = M;
-        cta_l[n] = den;
+      if (P == 1) {
+        const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
+        a.out[head * D + dd] = den > 0.f ? acc / den : 0.f;
+        if (dd == 0 && a.lse != nullptr)
+          a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
+      } else {
+        cta_o[n * D + dd] = acc;
+        if (dd == 0) {
+          cta_m[n] = M;
+          cta_l[n] = den;
+        }
       }
     }
-    cluster.sync();
-    // cluster combine: CTA cr finalises heads cr, cr + P, ...
-    for (int n = cr; n < a.R; n += P) {
-      for (int dd = tid; dd < D; dd += kRoutedThreads) {
+    if (P > 1) {
+      cluster.sync();
+      // cluster combine: CTA cr finalises heads cr, cr + P, ... (all (head, d)
+      // pairs of this CTA in parallel)
+      const int my_heads = cr < a.R ? (a.R - cr + P - 1) / P : 0;
+      for (int i = tid; i < my_heads * D; i += kRoutedThreads) {
+        const int n = cr + P * (i / D), dd = i % D;
         float M = -INFINITY;
         for (int pr = 0; pr < P; ++pr) M = fmaxf(M, cluster.map_shared_rank(cta_m, pr)[n]);
         float acc = 0.f, den = 0.f;
         if (M != -INFINITY) {
           for (int pr = 0; pr < P; ++pr) {
-            const float mp = cluster.map_shared_rank(cta_m, pr)[n];
-            if (mp == -INFINITY) continue;
-            const float f = ex2(mp - M);
+            const float f = ex2(cluster.map_shared_rank(cta_m, pr)[n] - M);  // -inf -> 0
             acc = fmaf(cluster.map_shared_rank(cta_o, pr)[n * D + dd], f, acc);
             den = fmaf(cluster.map_shared_rank(cta_l, pr)[n], f, den);
           }
@@ -449,8 +605,8 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
         if (dd == 0 && a.lse != nullptr)
           a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
       }
+      cluster.sync();
     }
-    cluster.sync();
   }
 }
 

@@ -34,7 +34,10 @@
  * Supported sizes: head_dim 64 or 128; n_q_heads % n_kv_heads == 0 with at most
  * 8 query heads per KV head; chunk % group == 0, chunk / group <= 32;
  * floor(max_len / chunk) <= 4096; 1 <= top_groups <= chunk / group;
- * top_chunks >= 1.
+ * top_chunks >= 1. Routing tables live in shared memory: parameter sets whose
+ * tables (about 4 * min(top_chunks, max_len/chunk) * (top_groups + chunk/group + 2)
+ * bytes) do not fit in shared memory next to the working buffers return
+ * HGA_ERR_UNSUPPORTED.
  */
 #ifndef HGA_H_
 #define HGA_H_
