@@ -61,6 +61,36 @@ def decode_bytes(L: int, w=W64) -> int:
             + S * hkv * d * 2 * 2 + hq * d * 2 + hq * d * 4 + hq * 4)
 
 
+def kernel_source_hash() -> str:
+    """sha256 (first 16 hex) of the kernel sources and the ABI header."""
+    import glob
+    import hashlib
+
+    files = sorted(glob.glob(os.path.join(ROOT, "hierarchical_routed_sparse_build_b200", "csrc", "*")))
+    files.append(os.path.join(ROOT, "include", "hga.h"))
+    h = hashlib.sha256()
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it covers these sources."""
+    import re
+
+    path = os.path.join(ROOT, "profiles", "decode_64k_routed_kernel.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -298,7 +328,9 @@ def run_gpu(args, rank: int, world: int, dist):
                    "ctas_per_head": args.ctas or "auto"},
         "roofline": {"bound": "hbm", "kernel": "routed_kernel<128, decode> (whole step, one launch)",
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": args.traffic,
+                     "frac": round(achieved / hbm, 4),
+                     "traffic": args.traffic if args.traffic is not None else
+                     (profiled_traffic() if B == 64 else None),
                      "alg_bytes_per_query": decode_bytes(w.ctx_len), "alg_bytes_per_launch": alg},
         "e2e": {"value": round(B * world * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_host.numel() * 2),

@@ -231,7 +231,7 @@ def test_routed_fraction_closed_form():
         assert len(np.unique(tok)) == S and np.all(np.diff(tok) > 0)
         assert tok[:128].tolist() == list(range(128))
         assert tok[-128:].tolist() == list(range((nf - 1) * 128, L))
-    # the pages' sparsity: about 3% at 64K
+    # the abstract's sparsity at 64K: roughly three percent
     assert 0.025 < rows[-1][3] / rows[-1][0] < 0.04
 
 
