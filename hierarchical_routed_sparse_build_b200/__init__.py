@@ -23,7 +23,8 @@ __all__ = [
     "HgaError", "hga_params", "hga_kv", "make_params", "make_kv", "library_path",
     "hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
-    "hga_status_string", "HGA_OPT_CTAS_PER_HEAD", "STATUS_NAMES", "EXPORTED",
+    "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
+    "hga_prefill", "HGA_OPT_CTAS_PER_HEAD", "STATUS_NAMES", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +36,8 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_UNSUPPORTED",
                 4: "HGA_ERR_DEVICE_FAULT", 5: "HGA_ERR_TIMEOUT"}
 EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
             "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
-            "hga_status_string")
+            "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
+            "hga_prefill")
 
 
 class HgaError(RuntimeError):
@@ -77,6 +79,10 @@ def _load() -> ctypes.CDLL:
         "hga_set_launch_option": ([i32, i32], i32),
         "hga_get_device_error": ([vp, ctypes.POINTER(i32)], i32),
         "hga_status_string": ([i32], ctypes.c_char_p),
+        "hga_route_blocks": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, i32, vp, vp], i32),
+        "hga_prefill_attend": ([vp, i32, i32, i32, KV, i32, vp, i32, vp, P, vp, vp], i32),
+        "hga_prefill_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
+        "hga_prefill": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -168,6 +174,35 @@ def hga_decode(q, n_q_heads: int, kv: hga_kv, chunk_sum, group_sum, p: hga_param
     _check(_lib.hga_decode(_addr(q), n_q_heads, ctypes.byref(kv), _addr(chunk_sum), _addr(group_sum),
                            ctypes.byref(p), _addr(out), _addr(lse), _addr(idx), idx_stride, _addr(n_idx),
                            _stream(stream)), "hga_decode")
+
+
+def hga_route_blocks(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int, chunk_sum,
+                     group_sum, p: hga_params, idx, idx_stride: int, n_idx, stream=None) -> None:
+    _check(_lib.hga_route_blocks(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
+                                 _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(idx), idx_stride,
+                                 _addr(n_idx), _stream(stream)), "hga_route_blocks")
+
+
+def hga_prefill_attend(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int, idx,
+                       idx_stride: int, n_idx, p: hga_params, out, stream=None) -> None:
+    _check(_lib.hga_prefill_attend(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len, _addr(idx),
+                                   idx_stride, _addr(n_idx), ctypes.byref(p), _addr(out), _stream(stream)),
+           "hga_prefill_attend")
+
+
+def hga_prefill_workspace_size(kv: hga_kv, n_q_heads: int, n_queries: int, block: int, cache_len: int,
+                               p: hga_params) -> int:
+    n = _lib.hga_prefill_workspace_size(ctypes.byref(kv), n_q_heads, n_queries, block, cache_len, ctypes.byref(p))
+    if n == 0:
+        raise HgaError(1, "hga_prefill_workspace_size")
+    return n
+
+
+def hga_prefill(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int, chunk_sum, group_sum,
+                p: hga_params, out, workspace, workspace_bytes: int, stream=None) -> None:
+    _check(_lib.hga_prefill(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len, _addr(chunk_sum),
+                            _addr(group_sum), ctypes.byref(p), _addr(out), _addr(workspace), workspace_bytes,
+                            _stream(stream)), "hga_prefill")
 
 
 def hga_set_launch_option(option: int, value: int) -> None:

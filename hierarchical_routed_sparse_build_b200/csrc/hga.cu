@@ -13,6 +13,8 @@
 
 #include "hga.h"
 #include "hga_common.cuh"
+#include "hga_prefill_attn.cuh"
+#include "hga_prefill_route.cuh"
 #include "hga_routed.cuh"
 #include "hga_summaries.cuh"
 
@@ -202,6 +204,105 @@ void routing_args(RoutedArgs& a, const hga_kv* kv, const hga_params* p) {
   a.kcap = kc < 1 ? 1 : kc;
 }
 
+// Routed tokens of one (block, head) when routing covers exactly [0, L).
+int routed_count(int L, const hga_params* p) {
+  const int C = p->chunk, nf = L / C;
+  if (nf <= 2) return L;
+  const int r = nf - 2 < p->top_chunks ? nf - 2 : p->top_chunks;
+  return C + r * p->top_groups * p->group + (L - (nf - 1) * C);
+}
+
+// Shared checks of the prefill calls (batch 1, contiguous cache, head dim 128,
+// blocks of 64 queries, 128-row tiles of two query heads).
+hga_status check_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block, const hga_kv* kv,
+                         int32_t cache_len, bool need_v) {
+  hga_status s = check_kv(kv, need_v);
+  if (s != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || n_queries < 1 || cache_len < 0) return HGA_ERR_INVALID_ARG;
+  if ((int64_t)cache_len + n_queries > kv->max_len) return HGA_ERR_INVALID_ARG;
+  if (kv->batch != 1 || kv->page_table != nullptr || kv->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+  if (block != kBlockQ || n_queries % block != 0) return HGA_ERR_UNSUPPORTED;
+  if (((n_q_heads / kv->n_kv_heads) * block) % kPfRows != 0) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+hga_status launch_block_route(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                              const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                              const hga_params* p, int32_t* idx, int32_t idx_stride, int32_t* n_idx,
+                              cudaStream_t stream) {
+  BlockRouteArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  a.T = n_queries;
+  a.block = block;
+  a.chunk_sum = static_cast<const uint16_t*>(chunk_sum);
+  a.group_sum = static_cast<const uint16_t*>(group_sum);
+  a.hkv = kv->n_kv_heads;
+  a.max_chunks = kv->max_len / p->chunk;
+  a.L = cache_len;
+  a.C = p->chunk;
+  a.g = p->group;
+  a.k = p->top_chunks;
+  a.G = p->top_groups;
+  a.idx = idx;
+  a.n_idx = n_idx;
+  a.idx_stride = idx_stride;
+  const int n_pad = a.max_chunks - 2 > 2 ? a.max_chunks - 2 : 2;
+  const int kcap_raw = a.max_chunks - 2 < a.k ? a.max_chunks - 2 : a.k;
+  const int kcap = kcap_raw < 1 ? 1 : kcap_raw;
+  const int smem = BlockRouteSmem(128, n_pad, kcap, a.G, a.C / a.g).total + 8 * n_pad;
+  if (smem > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
+  static std::atomic<int> smem_set[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
+  if (smem > smem_set[dev].load()) {
+    if (cudaFuncSetAttribute(block_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return HGA_ERR_CUDA;
+    smem_set[dev].store(smem);
+  }
+  const int units = (n_queries / block) * kv->n_kv_heads;
+  block_route_kernel<<<units, kRoutedThreads, smem, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                 const hga_kv* kv, int32_t cache_len, const int32_t* idx, int32_t idx_stride,
+                                 const int32_t* n_idx, const hga_params* p, float* out, cudaStream_t stream) {
+  PrefillAttnArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  a.T = n_queries;
+  a.block = block;
+  a.k = static_cast<const uint16_t*>(kv->k);
+  a.v = static_cast<const uint16_t*>(kv->v);
+  a.hkv = kv->n_kv_heads;
+  a.max_len = kv->max_len;
+  a.cache_len = cache_len;
+  a.idx = idx;
+  a.n_idx = n_idx;
+  a.idx_stride = idx_stride;
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.out = out;
+  static std::atomic<bool> configured[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
+  if (!configured[dev].load()) {
+    if (cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PrefillSmem::kTotal) != cudaSuccess)
+      return HGA_ERR_CUDA;
+    configured[dev].store(true);
+  }
+  const int m_tiles = a.R * block / kPfRows;
+  const int grid = (n_queries / block) * kv->n_kv_heads * m_tiles;
+  prefill_attn_kernel<<<grid, kPfThreads, PrefillSmem::kTotal, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace hga
 
@@ -343,6 +444,63 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
   a.n_idx_out = n_idx;
   a.idx_stride = idx ? idx_stride : 0;
   return run_routed<kModeDecode>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+hga_status hga_route_blocks(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                            const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                            const hga_params* p, int32_t* idx, int32_t idx_stride, int32_t* n_idx,
+                            cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, false);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+      idx == nullptr || n_idx == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if (idx_stride < routed_count(cache_len, p)) return HGA_ERR_INVALID_ARG;
+  return launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx,
+                            idx_stride, n_idx, stream);
+}
+
+hga_status hga_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                              const hga_kv* kv, int32_t cache_len, const int32_t* idx, int32_t idx_stride,
+                              const int32_t* n_idx, const hga_params* p, float* out, cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, false)) != HGA_OK) return s;
+  if (idx == nullptr || n_idx == nullptr || out == nullptr || idx_stride < 1) return HGA_ERR_INVALID_ARG;
+  return launch_prefill_attend(q, n_q_heads, n_queries, block, kv, cache_len, idx, idx_stride, n_idx, p, out,
+                               stream);
+}
+
+size_t hga_prefill_workspace_size(const hga_kv* kv, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                  int32_t cache_len, const hga_params* p) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK || block < 1 || n_queries < 1 ||
+      n_q_heads < 1 || cache_len < 0)
+    return 0;
+  const size_t units = (size_t)((n_queries + block - 1) / block) * kv->n_kv_heads;
+  const size_t stride = (size_t)routed_count(cache_len, p);
+  return units * (stride + 1) * sizeof(int32_t);
+}
+
+hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block, const hga_kv* kv,
+                       int32_t cache_len, const void* chunk_sum, const void* group_sum, const hga_params* p,
+                       float* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+      out == nullptr || workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return HGA_ERR_INVALID_ARG;
+  const size_t need = hga_prefill_workspace_size(kv, n_q_heads, n_queries, block, cache_len, p);
+  if (workspace_bytes < need) return HGA_ERR_INVALID_ARG;
+  const int stride = routed_count(cache_len, p);
+  const int units = (n_queries / block) * kv->n_kv_heads;
+  int32_t* idx = static_cast<int32_t*>(workspace);
+  int32_t* n_idx = idx + (size_t)units * stride;
+  s = launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx, stride,
+                         n_idx, stream);
+  if (s != HGA_OK) return s;
+  return launch_prefill_attend(q, n_q_heads, n_queries, block, kv, cache_len, idx, stride, n_idx, p, out, stream);
 }
 
 hga_status hga_set_launch_option(int32_t option, int32_t value) {

@@ -1,0 +1,252 @@
+// Block-shared two-level routing for chunked prefill.
+//
+// "Hierarchical Global Attention (HGA)", abstract (chunks, then groups, then
+// exact attention); the prefill reading: the queries of one block share a
+// routing decision whose chunk score is the maximum, over the block's queries,
+// of the head-summed score sum_i q_{p,i} . s_c (and likewise for groups).
+//
+// One CTA (kRoutedThreads) per (block, KV head). The scores form a small dense
+// product [n_q queries x D] . [D x chunks], computed on the tensor cores with
+// mma.sync m16n8k16: the fp32 head-summed queries are split into a bf16 high
+// part and a bf16 remainder (q = hi + lo, |lo| <= 2^-9 |q|), both multiplied by
+// the exact bf16 summaries and accumulated in fp32, which keeps the scores
+// within about 2^-16 relative of fp32 arithmetic. The maximum over the queries
+// is taken from the accumulator fragments (in-thread, then across the 8 lanes
+// that share a column). Top-k uses the same bucket select as decode.
+#pragma once
+
+#include "hga_common.cuh"
+#include "hga_routed.cuh"
+
+namespace hga {
+
+constexpr int kBlockQ = 64;  // queries per routing block (MMA M = 4 x 16)
+
+struct BlockRouteArgs {
+  const uint16_t* q;        // [T][Hq][D]
+  int hq, R, T, block;      // block == kBlockQ
+  const uint16_t* chunk_sum;  // [Hkv][max_chunks][D] (batch 1, contiguous)
+  const uint16_t* group_sum;  // [Hkv][max_chunks][gpc][D]
+  int hkv, max_chunks, L;     // L: cache length (routing covers [0, L))
+  int C, g, k, G;
+  int32_t* idx;    // [n_blocks][Hkv][idx_stride]
+  int32_t* n_idx;  // [n_blocks][Hkv]
+  int idx_stride;
+};
+
+// Shared memory of the block router (the launch adds 8 * n_pad bytes after
+// `total` for the bucket-select scratch).
+struct BlockRouteSmem {
+  int afrag, keys, sel, gmask, hist, misc, gsc, gstart, total;
+  __host__ __device__ static int up16(int x) { return (x + 15) & ~15; }
+  __host__ __device__ BlockRouteSmem(int D, int n_pad, int kcap, int gk, int gpc) {
+    int o = 0;
+    afrag = o;  o = up16(o + 4 * 8 * 2 * 32 * 16);  // [m-tile 4][k-step 8][hi/lo 2][lane 32] x uint4 (D = 128)
+    keys = o;   o = up16(o + 8 * n_pad);
+    sel = o;    o = up16(o + 4 * kcap);
+    gmask = o;  o = up16(o + 4 * kcap);
+    hist = o;   o = up16(o + 4 * kBuckets);
+    misc = o;   o = up16(o + 4 * 32);
+    gsc = o;    o = up16(o + 4 * kcap * gpc);
+    gstart = o; o = up16(o + 4 * kcap * gk);
+    total = o;
+    (void)D;
+  }
+};
+
+// Column maxima over the 64 queries of scores for 8 summary rows (one N tile).
+// The rows are the B operand: lane (g, t) passes the row of column g and loads
+// its units t + 4j, matching the permuted head-dim order of the A fragments
+// (see hga_attention.cuh). Returns, in lanes with g == 0, the maxima of columns
+// 2t and 2t+1.
+__device__ __forceinline__ void block_scores_tile(const uint4* afrag, const uint16_t* my_row, int lane,
+                                                  float& c0max, float& c1max) {
+  const int t = lane & 3;
+  uint4 bu[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bu[j] = ldg_nc(my_row + 8 * (t + 4 * j));
+  float acc[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int j = ks >> 1, p = ks & 1;
+    const uint32_t b0 = p ? bu[j].z : bu[j].x;
+    const uint32_t b1 = p ? bu[j].w : bu[j].y;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+      for (int hl = 0; hl < 2; ++hl) {
+        const uint4 a = afrag[((mt * 8 + ks) * 2 + hl) * 32 + lane];
+        mma_16816(acc[mt], a.x, a.y, a.z, a.w, b0, b1);
+      }
+    }
+  }
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    m0 = fmaxf(m0, fmaxf(acc[mt][0], acc[mt][2]));
+    m1 = fmaxf(m1, fmaxf(acc[mt][1], acc[mt][3]));
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, off));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, off));
+  }
+  c0max = m0;
+  c1max = m1;
+}
+
+__global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const BlockRouteArgs a) {
+  constexpr int D = 128;
+  extern __shared__ __align__(16) unsigned char br_smem[];
+  unsigned char* smem = br_smem;
+  const int blk = blockIdx.x / a.hkv, h = blockIdx.x % a.hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int W = kRoutedWarps;
+  const int gpc = a.C / a.g, gk = a.G;
+  const int nf = a.L / a.C;
+  const bool dense = nf <= 2;
+  const int n_cand = dense ? 0 : nf - 2;
+  const int r = n_cand < a.k ? n_cand : a.k;
+  const int n_pad = max(2, a.max_chunks - 2);
+  const int kcap = max(1, min(a.k, a.max_chunks - 2));
+  const BlockRouteSmem lay(D, n_pad, kcap, gk, gpc);
+  uint4* afrag = reinterpret_cast<uint4*>(smem + lay.afrag);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem + lay.keys);
+  int* sel = reinterpret_cast<int*>(smem + lay.sel);
+  uint32_t* gmask = reinterpret_cast<uint32_t*>(smem + lay.gmask);
+  int* hist = reinterpret_cast<int*>(smem + lay.hist);
+  int* misc = reinterpret_cast<int*>(smem + lay.misc);
+  float* gsc = reinterpret_cast<float*>(smem + lay.gsc);
+  int* gstart = reinterpret_cast<int*>(smem + lay.gstart);
+
+  // A fragments of the head-summed queries, hi/lo bf16 split, permuted head-dim
+  // order: fragment (m-tile mt, k-step ks = 2j+p) of lane (g, t): rows 16mt+g and
+  // 16mt+g+8, columns 8t + 32j + 4p + {0,1} (a0/a1) and + {2,3} (a2/a3).
+  const int q0 = blk * a.block;
+  for (int i = tid; i < 4 * 8 * 32; i += kRoutedThreads) {
+    const int l = i & 31, ks = (i >> 5) & 7, mt = i >> 8;
+    const int g = l >> 2, t = l & 3, j = ks >> 1, p = ks & 1;
+    const int col = 8 * t + 32 * j + 4 * p;
+    float v[2][4];  // [row g / g+8][col .. col+3]
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int qi = q0 + 16 * mt + g + 8 * rr;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float s = 0.f;
+        if (qi < a.T)
+          for (int hh = 0; hh < a.R; ++hh)
+            s += bf16_to_f(a.q[((int64_t)qi * a.hq + (int64_t)h * a.R + hh) * D + col + c]);
+        v[rr][c] = s;
+      }
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v[rr][c]));
+        const float h1 = __bfloat162float(__float2bfloat16_rn(v[rr][c + 1]));
+        // register order: a0 = (row g, cols c0,c1), a1 = (row g+8, c0,c1), a2 = (g, c2,c3), a3 = (g+8, c2,c3)
+        const int reg = (c >> 1) * 2 + rr;
+        hi[reg] = pack_bf16x2(h0, h1);
+        lo[reg] = pack_bf16x2(v[rr][c] - h0, v[rr][c + 1] - h1);
+      }
+    afrag[((mt * 8 + ks) * 2 + 0) * 32 + l] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    afrag[((mt * 8 + ks) * 2 + 1) * 32 + l] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  for (int i = tid; i < n_pad; i += kRoutedThreads) keys[i] = 0ull;
+  __syncthreads();
+
+  const uint16_t* cs = a.chunk_sum + (int64_t)h * a.max_chunks * D;
+  const uint16_t* gs = a.group_sum + (int64_t)h * a.max_chunks * gpc * D;
+  // chunk scores, 8 candidates per warp tile
+  if (n_cand > r) {
+    const int n_tiles = (n_cand + 7) / 8;
+    for (int tile = warp; tile < n_tiles; tile += W) {
+      const uint16_t* my_row = cs + (int64_t)(min(tile * 8 + (lane >> 2), n_cand - 1) + 1) * D;
+      float m0, m1;
+      block_scores_tile(afrag, my_row, lane, m0, m1);
+      if ((lane >> 2) == 0) {
+        const int t4 = lane & 3;
+        const int ca = tile * 8 + 2 * t4, cb = ca + 1;
+        if (ca < n_cand) keys[ca] = route_key(m0, (uint32_t)(ca + 1));
+        if (cb < n_cand) keys[cb] = route_key(m1, (uint32_t)(cb + 1));
+      }
+    }
+    __syncthreads();
+    // scratch for the boundary bucket: n_pad keys right after the layout
+    select_top_chunks(keys, n_cand, r, sel, hist, misc, reinterpret_cast<uint64_t*>(smem + lay.total), n_pad);
+  } else {
+    for (int i = tid; i < r; i += kRoutedThreads) sel[i] = i + 1;
+  }
+  __syncthreads();
+
+  // group scores: one kept chunk (gpc rows, <= 32) per warp tile of 8 rows
+  const bool all_groups = gk >= gpc;
+  if (!all_groups) {
+    const int tiles_per_chunk = (gpc + 7) / 8;
+    for (int wt = warp; wt < r * tiles_per_chunk; wt += W) {
+      const int ci = wt / tiles_per_chunk, part = wt - ci * tiles_per_chunk;
+      const uint16_t* my_row = gs + ((int64_t)sel[ci] * gpc + min(part * 8 + (lane >> 2), gpc - 1)) * D;
+      float m0, m1;
+      block_scores_tile(afrag, my_row, lane, m0, m1);
+      if ((lane >> 2) == 0) {
+        const int t4 = lane & 3;
+        const int ja = part * 8 + 2 * t4, jb = ja + 1;
+        if (ja < gpc) gsc[ci * gpc + ja] = m0;
+        if (jb < gpc) gsc[ci * gpc + jb] = m1;
+      }
+    }
+    for (int i = tid; i < r; i += kRoutedThreads) gmask[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < r * gpc; i += kRoutedThreads) {
+      const int ci = i / gpc, j = i - ci * gpc;
+      const float tj = gsc[i];
+      int rank = 0;
+      for (int l = 0; l < gpc; ++l) {
+        const float tl = gsc[ci * gpc + l];
+        rank += (tl > tj) || (tl == tj && l < j);
+      }
+      if (rank < gk) atomicOr(&gmask[ci], 1u << j);
+    }
+    __syncthreads();
+  }
+  const uint32_t full_mask = gpc >= 32 ? 0xFFFFFFFFu : ((1u << gpc) - 1u);
+  for (int i = tid; i < r; i += kRoutedThreads) {
+    uint32_t m = all_groups ? full_mask : gmask[i];
+    for (int qq = 0; qq < gk; ++qq) {
+      const int j = m ? __ffs(m) - 1 : 0;
+      m &= m - 1;
+      gstart[i * gk + qq] = sel[i] * a.C + j * a.g;
+    }
+  }
+  __syncthreads();
+  const int S = dense ? a.L : a.C + r * gk * a.g + (a.L - (nf - 1) * a.C);
+  const int unit = blk * a.hkv + h;
+  const int span = gk * a.g;
+  const int Sw = min(S, a.idx_stride);
+  if (S > a.idx_stride && tid == 0) report_error(kErrIndex);
+  for (int e = tid; e < Sw; e += kRoutedThreads) {
+    int tok;
+    if (dense || e < a.C) {
+      tok = e;
+    } else {
+      const int u = e - a.C;
+      if (u < r * span) {
+        const int i = u / span, rem = u - i * span, qq = rem / a.g;
+        tok = gstart[i * gk + qq] + (rem - qq * a.g);
+      } else {
+        tok = (nf - 1) * a.C + (u - r * span);
+      }
+    }
+    a.idx[(int64_t)unit * a.idx_stride + e] = tok;
+  }
+  if (tid == 0) a.n_idx[unit] = Sw;
+}
+
+}  // namespace hga

@@ -172,6 +172,60 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
                       int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream);
 
 /*
+ * Chunked prefill. n_queries new tokens sit at positions cache_len ..
+ * cache_len + n_queries - 1; their keys and values are already written into
+ * the cache at those positions (kv->max_len >= cache_len + n_queries). The
+ * queries are cut into blocks of `block` consecutive queries. Supported: batch 1,
+ * contiguous cache, head_dim 128, block 64, n_queries % block == 0, and an even
+ * number of query heads per KV head (two heads x 64 queries per 128-row tile).
+ * kv->seq_lens is not read by the prefill calls; cache_len is given directly.
+ * Summaries must cover the cache's full chunks (hga_build_summaries with
+ * seq_lens[0] = cache_len).
+ *
+ * Block-shared routing (the prefill reading of the abstract's two-level
+ * routing): for block b and KV head h, chunk scores are
+ *   sigma_c = max over the block's queries p of sum_i q_{p,i} . s_c
+ * and group scores likewise; the kept chunks, groups, sink and local chunk of
+ * the cache [0, cache_len) follow hga_route. The scores are computed on tensor
+ * cores with the head-summed queries split into a bf16 high part and a bf16
+ * remainder (about 2^-16 relative error).
+ *   idx   [n_queries/block][n_kv_heads][idx_stride] int32 out: routed cache positions
+ *   n_idx [n_queries/block][n_kv_heads] int32 out
+ * idx_stride must be >= the routed count for cache_len (hga_max_routed_tokens
+ * of a cache with max_len = cache_len bounds it).
+ */
+hga_status hga_route_blocks(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                            const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                            const hga_params* p, int32_t* idx, int32_t idx_stride, int32_t* n_idx,
+                            cudaStream_t stream);
+
+/*
+ * Prefill attention over given routed cache sets (abstract: exact attention over
+ * the retrieved tokens): query p of block b (position P + p, P = cache_len + 64 b)
+ * attends, for each of its query heads, to the cache positions idx[b][h][0:n_idx]
+ * plus the block's own positions P .. P + p. Tensor-core (tcgen05) contraction
+ * with fp32 accumulation in tensor memory.
+ *   q [n_queries][n_q_heads][128] bf16, out [n_queries][n_q_heads][128] float32.
+ * Only p->scale is read from p.
+ */
+hga_status hga_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                              const hga_kv* kv, int32_t cache_len, const int32_t* idx, int32_t idx_stride,
+                              const int32_t* n_idx, const hga_params* p, float* out, cudaStream_t stream);
+
+/* Bytes of workspace hga_prefill needs (0 on invalid arguments). */
+size_t hga_prefill_workspace_size(const hga_kv* kv, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                  int32_t cache_len, const hga_params* p);
+
+/*
+ * hga_route_blocks followed by hga_prefill_attend; the routed lists live in the
+ * caller's workspace (device memory, 4-byte aligned, at least
+ * hga_prefill_workspace_size bytes; its contents on return are unspecified).
+ */
+hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block, const hga_kv* kv,
+                       int32_t cache_len, const void* chunk_sum, const void* group_sum, const hga_params* p,
+                       float* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Launch tuning, process-wide (not thread-safe against concurrent calls).
  *   HGA_OPT_CTAS_PER_HEAD: CTAs (one thread-block cluster) that cooperate on one
  *   (sequence, KV head) in hga_route / hga_attend / hga_decode; 0 = automatic,
