@@ -24,7 +24,7 @@ __all__ = [
     "hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
-    "hga_prefill", "HGA_OPT_CTAS_PER_HEAD", "STATUS_NAMES", "EXPORTED",
+    "hga_prefill", "hga_prefill_noalloc", "HGA_OPT_CTAS_PER_HEAD", "STATUS_NAMES", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,7 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_UNSUPPORTED",
 EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
             "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
             "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
-            "hga_prefill")
+            "hga_prefill", "hga_prefill_noalloc")
 
 
 class HgaError(RuntimeError):
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "hga_prefill_attend": ([vp, i32, i32, i32, KV, i32, vp, i32, vp, P, vp, vp], i32),
         "hga_prefill_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
         "hga_prefill": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
+        "hga_prefill_noalloc": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -203,6 +204,15 @@ def hga_prefill(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache
     _check(_lib.hga_prefill(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len, _addr(chunk_sum),
                             _addr(group_sum), ctypes.byref(p), _addr(out), _addr(workspace), workspace_bytes,
                             _stream(stream)), "hga_prefill")
+
+
+def hga_prefill_noalloc(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int, chunk_sum,
+                        group_sum, p: hga_params, out, stream=None) -> None:
+    """hga_prefill without a workspace, for callers that cannot allocate device memory
+    (the routed lists live in a 2 MiB array inside the library; see hga.h)."""
+    _check(_lib.hga_prefill_noalloc(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
+                                    _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(out),
+                                    _stream(stream)), "hga_prefill_noalloc")
 
 
 def hga_set_launch_option(option: int, value: int) -> None:

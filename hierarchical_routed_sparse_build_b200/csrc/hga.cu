@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <climits>
+#include <mutex>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -303,6 +304,31 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
   return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
 }
 
+// Routed-list area of hga_prefill_noalloc: a fixed device array that every GPU
+// loading the library keeps until process exit, so that the entry point never
+// allocates. Host code must not pass the symbol itself to a kernel (on the host
+// it is only a stand-in); the device address comes from cudaGetSymbolAddress.
+constexpr size_t kNoAllocPrefillBytes = 2u << 20;
+static __device__ __align__(256) unsigned char g_noalloc_prefill_ws[kNoAllocPrefillBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_prefill_ws on the current device, looked up once
+// per device (with that device current) and cached.
+hga_status noalloc_area(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_prefill_ws) != cudaSuccess || ptr == nullptr) return HGA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HGA_OK;
+}
+
 }  // namespace
 }  // namespace hga
 
@@ -496,6 +522,31 @@ hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int3
   const int stride = routed_count(cache_len, p);
   const int units = (n_queries / block) * kv->n_kv_heads;
   int32_t* idx = static_cast<int32_t*>(workspace);
+  int32_t* n_idx = idx + (size_t)units * stride;
+  s = launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx, stride,
+                         n_idx, stream);
+  if (s != HGA_OK) return s;
+  return launch_prefill_attend(q, n_q_heads, n_queries, block, kv, cache_len, idx, stride, n_idx, p, out, stream);
+}
+
+hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                               const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                               const hga_params* p, float* out, cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+      out == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if (hga_prefill_workspace_size(kv, n_q_heads, n_queries, block, cache_len, p) > kNoAllocPrefillBytes)
+    return HGA_ERR_UNSUPPORTED;
+  void* area = nullptr;
+  if ((s = noalloc_area(&area)) != HGA_OK) return s;
+  // Every list entry read later is written first by the routing kernel, so the
+  // area needs no clearing between calls.
+  const int stride = routed_count(cache_len, p);
+  const int units = (n_queries / block) * kv->n_kv_heads;
+  int32_t* idx = static_cast<int32_t*>(area);
   int32_t* n_idx = idx + (size_t)units * stride;
   s = launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx, stride,
                          n_idx, stream);

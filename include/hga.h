@@ -22,8 +22,9 @@
  *   - bfloat16 tensors are passed as raw 16-bit patterns (`const void*`), 16-byte
  *     aligned; int32/float tensors are naturally aligned.
  *   - Calls are asynchronous on `stream`. The library allocates no device
- *     memory; its only state is one device error word per device (a __device__
- *     variable) and a process-wide launch option (hga_set_launch_option).
+ *     memory; its state is one device error word per device (a __device__
+ *     variable), the fixed routed-list array of hga_prefill_noalloc, and a
+ *     process-wide launch option (hga_set_launch_option).
  *   - Host validation failures return HGA_ERR_INVALID_ARG or
  *     HGA_ERR_UNSUPPORTED synchronously with nothing enqueued. Problems only the
  *     device can see (a sequence length above max_len, a page id outside the
@@ -224,6 +225,31 @@ size_t hga_prefill_workspace_size(const hga_kv* kv, int32_t n_q_heads, int32_t n
 hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block, const hga_kv* kv,
                        int32_t cache_len, const void* chunk_sum, const void* group_sum, const hga_params* p,
                        float* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * hga_prefill for callers that cannot allocate device memory. (The paper has no
+ * counterpart; this is a property of the library.) Some callers have no way to
+ * hand the library a workspace: a plugin whose host framework owns every device
+ * allocation and gives the plugin no allocator, or a caller that must keep
+ * cudaMalloc (which may synchronise the device) out of its serving loop. This
+ * entry point allocates nothing and takes no workspace: the routed lists go to a
+ * 2 MiB array of device memory inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *   - Same arguments and results as hga_prefill, without the workspace.
+ *   - Limit: hga_prefill_workspace_size(...) must be at most 2 MiB (for example
+ *     2048 queries in blocks of 64 with 4 KV heads and 2304 routed tokens uses
+ *     1.18 MB); larger problems return HGA_ERR_UNSUPPORTED with nothing enqueued.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents (nothing in it needs clearing: every entry that is read is
+ *     written first by the same call). Calls whose execution overlaps on the GPU
+ *     (different streams without ordering) race on it: order them.
+ */
+hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                               const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                               const hga_params* p, float* out, cudaStream_t stream);
 
 /*
  * Launch tuning, process-wide (not thread-safe against concurrent calls).
