@@ -91,6 +91,89 @@ def profiled_traffic():
     return int(m_bytes.group(1))
 
 
+def bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
+def prefill_flops(keys_per_block: int, w=synth.PREFILL_64K) -> int:
+    """QK^T and PV flops of a prefill: every (query, head) against its block's keys."""
+    return 2 * 2 * (w.n_new * w.n_q_heads) * keys_per_block * w.head_dim
+
+
+def run_prefill(dev, steps: int, warmup: int):
+    """Time hga_prefill on the 2048-new-token, 63488-token-cache workload."""
+    import torch
+
+    import hierarchical_routed_sparse_build_b200 as hga
+    import oracle
+
+    w = synth.PREFILL_64K
+    inp = synth.prefill_inputs(w)
+    L0, T = inp.cache_len, w.n_new
+    dv = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    k, v, q = dv(inp.k), dv(inp.v), dv(inp.q)
+    lens = torch.tensor([L0], dtype=torch.int32, device=dev)
+    kv = hga.make_kv(k, v, lens, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, max_len=k.shape[2], batch=1)
+    p = hga.make_params(w.chunk, w.group, w.top_chunks, w.top_groups)
+    nc = k.shape[2] // w.chunk
+    cs = torch.zeros((1, w.n_kv_heads, nc, w.head_dim), dtype=torch.bfloat16, device=dev)
+    gs = torch.zeros((1, w.n_kv_heads, nc, w.chunk // w.group, w.head_dim), dtype=torch.bfloat16, device=dev)
+    hga.hga_build_summaries(kv, p, cs, gs)
+    wsb = hga.hga_prefill_workspace_size(kv, w.n_q_heads, T, w.block, L0, p)
+    ws = torch.zeros(wsb // 4, dtype=torch.int32, device=dev)
+    stride = oracle.max_routed(L0, w.chunk, w.group, w.top_chunks, w.top_groups)
+    nb = T // w.block
+    idx = ws[: nb * w.n_kv_heads * stride].view(nb, w.n_kv_heads, stride)
+    n_idx = ws[nb * w.n_kv_heads * stride: nb * w.n_kv_heads * (stride + 1)].view(nb, w.n_kv_heads)
+    out = torch.empty((T, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.max()
+            st[i].record(stream)
+            fn()
+            en[i].record(stream)
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in zip(st, en)])
+
+    full = timed(lambda: hga.hga_prefill(q, w.n_q_heads, T, w.block, kv, L0, cs, gs, p, out, ws, wsb), steps)
+    route = timed(lambda: hga.hga_route_blocks(q, w.n_q_heads, T, w.block, kv, L0, cs, gs, p, idx, stride,
+                                               n_idx), steps)
+    attend = timed(lambda: hga.hga_prefill_attend(q, w.n_q_heads, T, w.block, kv, L0, idx, stride, n_idx, p,
+                                                  out), steps)
+    st, bits = hga.hga_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in prefill: {bits}")
+    keys = int(n_idx.sum().item()) // (nb * w.n_kv_heads) + w.block
+    fl = prefill_flops(keys)
+    burst, sustained, kind = bf16_peak()
+    attn_tf = fl / (attend * 1e-3) / 1e12
+    return {
+        "workload": "prefill_2048_on_63488: 2048 new tokens in 32 blocks of 64 on a 63488-token cache, 32 q / "
+                    "4 KV heads, d 128, block-shared routing (C 128, g 16, top-32 + sink + local, top-4 groups) "
+                    "+ own causal block; 2368 keys per block",
+        "tokens_per_s": round(T / (full * 1e-3), 1), "ms_per_step": round(full, 4),
+        "route_ms": round(route, 4), "attend_ms": round(attend, 4),
+        "flops_per_step": fl, "tflops_step": round(fl / (full * 1e-3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel (tcgen05, TMEM accumulators)",
+                     "achieved": round(attn_tf, 1), "peak": burst, "peak_kind": f"{kind} bf16 burst",
+                     "unit": "TFLOP/s", "frac": round(attn_tf / burst, 4),
+                     "frac_of_sustained": round(attn_tf / sustained, 4)},
+    }
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -315,6 +398,7 @@ def run_gpu(args, rank: int, world: int, dist):
     achieved = alg / mean_launch_s / 1e9
     srt = sorted(times)
     pct = lambda p: srt[min(len(srt) - 1, int(round(p / 100 * (len(srt) - 1))))]
+    prefill = None if args.no_prefill else run_prefill(dev, max(5, args.steps // 10), args.warmup)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -340,6 +424,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "latency_ms": {"p50": round(pct(50), 5), "p95": round(pct(95), 5), "p99": round(pct(99), 5)},
         "batch1_latency_us": round(statistics.median(lat) * 1e3, 2),
         "sweep": sweep,
+        "prefill": prefill,
     }
     return res, inp, w
 
@@ -356,6 +441,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None, help="ncu dram bytes per launch, if measured")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

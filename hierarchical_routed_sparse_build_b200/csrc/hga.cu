@@ -296,6 +296,11 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
     if (cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PrefillSmem::kTotal) != cudaSuccess)
       return HGA_ERR_CUDA;
+    // two CTAs per SM need the largest shared-memory carveout; this kernel
+    // moves K/V with cp.async into shared memory, so a small L1 costs nothing
+    if (cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+        cudaSuccess)
+      return HGA_ERR_CUDA;
     configured[dev].store(true);
   }
   const int m_tiles = a.R * block / kPfRows;

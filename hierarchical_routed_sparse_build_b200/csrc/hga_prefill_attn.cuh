@@ -97,18 +97,16 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
   const int32_t* ilist = a.idx + (int64_t)unit * a.idx_stride;
   const int64_t head_row0 = (int64_t)h * a.max_len;
 
-  // key entry -> row of K/V (padding repeats entry 0's row; it is masked)
-  auto key_row = [&](int e) -> int64_t {
-    int tok;
-    if (e < n_cache) {
-      tok = __ldg(ilist + e);
-      if (tok < 0 || tok >= a.cache_len) {
-        report_error(kErrIndex);
-        tok = own0;
-      }
-    } else if (e < n_keys) {
-      tok = own0 + (e - n_cache);
-    } else {
+  // Key entry e -> token, in two steps so that the list is read one tile ahead
+  // without waiting for the load: raw_token() only loads (cache entries), and
+  // key_row() validates and turns the token into a K/V row when the copies are
+  // issued. Padding entries repeat the block's first own token; they are masked.
+  auto raw_token = [&](int e) -> int {
+    return e < n_cache ? __ldg(ilist + e) : (e < n_keys ? own0 + (e - n_cache) : own0);
+  };
+  auto key_row = [&](int e, int tok) -> int64_t {
+    if (e < n_cache && (tok < 0 || tok >= a.cache_len)) {
+      report_error(kErrIndex);
       tok = own0;
     }
     return head_row0 + tok;
@@ -122,19 +120,32 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     const int64_t row = (int64_t)(blk * a.block + pp) * a.hq + (int64_t)h * a.R + hl;
     cp_async16(sQ + (u >> 3) * 16384 + sw128(rr, u & 7), a.q + row * D + 8 * u);
   }
-  auto issue_tile = [&](int j, int st) {
+  // Thread tid copies unit (tid % 16) of keys tid/16 + 8i (i < 8) of a tile: 16
+  // consecutive threads cover one 256-byte row. All eight row lookups are
+  // issued before the first copy (the copies are ordered memory operations).
+  const int cu = tid & 15, ck = tid >> 4;
+  auto tile_tokens = [&](int j, int (&tok)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tok[i] = raw_token(j * kPfKeys + ck + 8 * i);
+  };
+  auto issue_tile = [&](int j, const int (&tok)[8], int st) {
     unsigned char* sK = smem + PrefillSmem::kK + st * 16384;
     unsigned char* sV = smem + PrefillSmem::kV + st * 16384;
-    for (int i = tid; i < kPfKeys * 16; i += kPfThreads) {
-      const int c = i >> 4, u = i & 15;
-      const int64_t row = key_row(j * kPfKeys + c);
-      const uint32_t off = (u >> 3) * 8192 + sw128(c, u & 7);
-      cp_async16(sK + off, a.k + row * D + 8 * u);
-      cp_async16(sV + off, a.v + row * D + 8 * u);
+    int64_t rows[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rows[i] = key_row(j * kPfKeys + ck + 8 * i, tok[i]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t off = (cu >> 3) * 8192 + sw128(ck + 8 * i, cu & 7);
+      cp_async16(sK + off, a.k + rows[i] * D + 8 * cu);
+      cp_async16(sV + off, a.v + rows[i] * D + 8 * cu);
     }
   };
-  issue_tile(0, 0);
+  int next_tok[8];
+  tile_tokens(0, next_tok);
+  issue_tile(0, next_tok, 0);
   cp_async_commit();
+  if (n_tiles > 1) tile_tokens(1, next_tok);
 
   if (tid == 0) {
     mbar_init(bar_s, 1);
@@ -178,25 +189,36 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     }
     // stage j-1 is free once PV_{j-1} has completed; then prefetch tile j+1 into it
     if (j >= 1 && !mbar_wait_bounded(bar_o, (uint32_t)((j - 1) & 1))) ok = false;
-    if (j + 1 < n_tiles) issue_tile(j + 1, st ^ 1);
+    if (j + 1 < n_tiles) issue_tile(j + 1, next_tok, st ^ 1);
     cp_async_commit();
+    if (j + 2 < n_tiles) tile_tokens(j + 2, next_tok);  // list entries of the tile after next
     if (!mbar_wait_bounded(bar_s, (uint32_t)(j & 1))) ok = false;
     tc_fence_after();
 
-    // softmax of this thread's row
+    // softmax of this thread's row; only tiles reaching past the routed cache
+    // entries need a mask (the block's own tokens are causal, the rest is padding)
     uint32_t sv[2][32];
     tmem_ld32(tS + lane_off + 0, sv[0]);
     tmem_ld32(tS + lane_off + 32, sv[1]);
     tmem_wait_ld();
-    float x[kPfKeys];
-    float tmax = -INFINITY;
+    const bool masked_tile = (j + 1) * kPfKeys > n_cache;
+    if (masked_tile) {
 #pragma unroll
-    for (int c = 0; c < kPfKeys; ++c) {
-      const int e = j * kPfKeys + c;
-      const bool valid = e < n_cache || (e < n_keys && (e - n_cache) <= p);
-      x[c] = valid ? __uint_as_float(sv[c >> 5][c & 31]) * sl : -INFINITY;
-      tmax = fmaxf(tmax, x[c]);
+      for (int c = 0; c < kPfKeys; ++c) {
+        const int e = j * kPfKeys + c;
+        const bool valid = e < n_cache || (e < n_keys && (e - n_cache) <= p);
+        if (!valid) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+      }
     }
+    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      mx0 = fmaxf(mx0, __uint_as_float(sv[0][c]));
+      mx1 = fmaxf(mx1, __uint_as_float(sv[0][c + 1]));
+      mx2 = fmaxf(mx2, __uint_as_float(sv[1][c]));
+      mx3 = fmaxf(mx3, __uint_as_float(sv[1][c + 1]));
+    }
+    const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;  // sl > 0
     const bool need = tmax > m_ref + kRescaleLog2 || (m_ref == -INFINITY && tmax != -INFINITY);
     float alpha = 1.f;
     if (need) {
@@ -217,16 +239,18 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
       }
       tmem_wait_st();
     }
-    const float base = m_ref == -INFINITY ? 0.f : m_ref;
+    const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
     unsigned char* sP = smem + PrefillSmem::kP;
+    float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       float pv[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        pv[c] = ex2(x[8 * u + c] - base);
-        l_sum += pv[c];
-      }
+      for (int c = 0; c < 8; ++c) pv[c] = ex2(fmaf(__uint_as_float(sv[u >> 2][8 * (u & 3) + c]), sl, nbase));
+      ls0 += pv[0] + pv[4];
+      ls1 += pv[1] + pv[5];
+      ls2 += pv[2] + pv[6];
+      ls3 += pv[3] + pv[7];
       uint4 w;
       w.x = pack_bf16x2(pv[0], pv[1]);
       w.y = pack_bf16x2(pv[2], pv[3]);
@@ -234,6 +258,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
       w.w = pack_bf16x2(pv[6], pv[7]);
       *reinterpret_cast<uint4*>(sP + sw128(r, u)) = w;
     }
+    l_sum += (ls0 + ls1) + (ls2 + ls3);
     if (!ok) *abort_flag = 1;
     fence_async_smem();
     tc_fence_before();

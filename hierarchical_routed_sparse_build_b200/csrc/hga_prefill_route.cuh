@@ -37,11 +37,12 @@ struct BlockRouteArgs {
 // Shared memory of the block router (the launch adds 8 * n_pad bytes after
 // `total` for the bucket-select scratch).
 struct BlockRouteSmem {
-  int afrag, keys, sel, gmask, hist, misc, gsc, gstart, total;
+  int afrag, qs, keys, sel, gmask, hist, misc, gsc, gstart, total;
   __host__ __device__ static int up16(int x) { return (x + 15) & ~15; }
   __host__ __device__ BlockRouteSmem(int D, int n_pad, int kcap, int gk, int gpc) {
     int o = 0;
     afrag = o;  o = up16(o + 4 * 8 * 2 * 32 * 16);  // [m-tile 4][k-step 8][hi/lo 2][lane 32] x uint4 (D = 128)
+    qs = o;     o = up16(o + 4 * kBlockQ * D);       // head-summed queries, fp32 [64][D]
     keys = o;   o = up16(o + 8 * n_pad);
     sel = o;    o = up16(o + 4 * kcap);
     gmask = o;  o = up16(o + 4 * kcap);
@@ -55,22 +56,24 @@ struct BlockRouteSmem {
 };
 
 // Column maxima over the 64 queries of scores for 8 summary rows (one N tile).
-// The rows are the B operand: lane (g, t) passes the row of column g and loads
-// its units t + 4j, matching the permuted head-dim order of the A fragments
-// (see hga_attention.cuh). Returns, in lanes with g == 0, the maxima of columns
-// 2t and 2t+1.
-__device__ __forceinline__ void block_scores_tile(const uint4* afrag, const uint16_t* my_row, int lane,
-                                                  float& c0max, float& c1max) {
+// The rows are the B operand: lane (g, t) holds units t + 4j of the row of column
+// g (load_b_units), matching the permuted head-dim order of the A fragments (see
+// hga_attention.cuh). Returns, in lanes with g == 0, the maxima of columns 2t
+// and 2t+1. Callers load the next tile's units before scoring the current one.
+__device__ __forceinline__ void load_b_units(const uint16_t* my_row, int lane, uint4 (&bu)[4]) {
   const int t = lane & 3;
-  uint4 bu[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) bu[j] = ldg_nc(my_row + 8 * (t + 4 * j));
+}
+
+__device__ __forceinline__ void block_scores_tile(const uint4* afrag, const uint4 (&bu)[4], int lane,
+                                                  float& c0max, float& c1max) {
   float acc[4][4];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-#pragma unroll
+#pragma unroll 2
   for (int ks = 0; ks < 8; ++ks) {
     const int j = ks >> 1, p = ks & 1;
     const uint32_t b0 = p ? bu[j].z : bu[j].x;
@@ -123,27 +126,37 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
   float* gsc = reinterpret_cast<float*>(smem + lay.gsc);
   int* gstart = reinterpret_cast<int*>(smem + lay.gstart);
 
+  // Head-summed queries of the block (fp32, 16-byte loads of 8 head dims).
+  float* qs = reinterpret_cast<float*>(smem + lay.qs);
+  const int q0 = blk * a.block;
+  for (int i = tid; i < kBlockQ * (D / 8); i += kRoutedThreads) {
+    const int row = i / (D / 8), u = i - row * (D / 8);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int qi = q0 + row;
+    if (qi < a.T) {
+      const uint16_t* base = a.q + ((int64_t)qi * a.hq + (int64_t)h * a.R) * D + 8 * u;
+      for (int hh = 0; hh < a.R; ++hh) {
+        const uint4 v = ldg_nc(base + (int64_t)hh * D);
+        acc[0] += bf16_lo(v.x); acc[1] += bf16_hi(v.x); acc[2] += bf16_lo(v.y); acc[3] += bf16_hi(v.y);
+        acc[4] += bf16_lo(v.z); acc[5] += bf16_hi(v.z); acc[6] += bf16_lo(v.w); acc[7] += bf16_hi(v.w);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) qs[row * D + 8 * u + c] = acc[c];
+  }
+  __syncthreads();
   // A fragments of the head-summed queries, hi/lo bf16 split, permuted head-dim
   // order: fragment (m-tile mt, k-step ks = 2j+p) of lane (g, t): rows 16mt+g and
   // 16mt+g+8, columns 8t + 32j + 4p + {0,1} (a0/a1) and + {2,3} (a2/a3).
-  const int q0 = blk * a.block;
   for (int i = tid; i < 4 * 8 * 32; i += kRoutedThreads) {
     const int l = i & 31, ks = (i >> 5) & 7, mt = i >> 8;
     const int g = l >> 2, t = l & 3, j = ks >> 1, p = ks & 1;
     const int col = 8 * t + 32 * j + 4 * p;
     float v[2][4];  // [row g / g+8][col .. col+3]
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int qi = q0 + 16 * mt + g + 8 * rr;
+    for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float s = 0.f;
-        if (qi < a.T)
-          for (int hh = 0; hh < a.R; ++hh)
-            s += bf16_to_f(a.q[((int64_t)qi * a.hq + (int64_t)h * a.R + hh) * D + col + c]);
-        v[rr][c] = s;
-      }
-    }
+      for (int c = 0; c < 4; ++c) v[rr][c] = qs[(16 * mt + g + 8 * rr) * D + col + c];
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr)
@@ -167,10 +180,15 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
   // chunk scores, 8 candidates per warp tile
   if (n_cand > r) {
     const int n_tiles = (n_cand + 7) / 8;
+    auto row_of = [&](int tile) { return cs + (int64_t)(min(tile * 8 + (lane >> 2), n_cand - 1) + 1) * D; };
+    uint4 bu[4], bn[4];
+    if (warp < n_tiles) load_b_units(row_of(warp), lane, bu);
     for (int tile = warp; tile < n_tiles; tile += W) {
-      const uint16_t* my_row = cs + (int64_t)(min(tile * 8 + (lane >> 2), n_cand - 1) + 1) * D;
+      if (tile + W < n_tiles) load_b_units(row_of(tile + W), lane, bn);
       float m0, m1;
-      block_scores_tile(afrag, my_row, lane, m0, m1);
+      block_scores_tile(afrag, bu, lane, m0, m1);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bu[j] = bn[j];
       if ((lane >> 2) == 0) {
         const int t4 = lane & 3;
         const int ca = tile * 8 + 2 * t4, cb = ca + 1;
@@ -190,11 +208,20 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
   const bool all_groups = gk >= gpc;
   if (!all_groups) {
     const int tiles_per_chunk = (gpc + 7) / 8;
-    for (int wt = warp; wt < r * tiles_per_chunk; wt += W) {
+    auto grow_of = [&](int wt) {
       const int ci = wt / tiles_per_chunk, part = wt - ci * tiles_per_chunk;
-      const uint16_t* my_row = gs + ((int64_t)sel[ci] * gpc + min(part * 8 + (lane >> 2), gpc - 1)) * D;
+      return gs + ((int64_t)sel[ci] * gpc + min(part * 8 + (lane >> 2), gpc - 1)) * D;
+    };
+    const int n_gt = r * tiles_per_chunk;
+    uint4 bu[4], bn[4];
+    if (warp < n_gt) load_b_units(grow_of(warp), lane, bu);
+    for (int wt = warp; wt < n_gt; wt += W) {
+      const int ci = wt / tiles_per_chunk, part = wt - ci * tiles_per_chunk;
+      if (wt + W < n_gt) load_b_units(grow_of(wt + W), lane, bn);
       float m0, m1;
-      block_scores_tile(afrag, my_row, lane, m0, m1);
+      block_scores_tile(afrag, bu, lane, m0, m1);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bu[j] = bn[j];
       if ((lane >> 2) == 0) {
         const int t4 = lane & 3;
         const int ja = part * 8 + 2 * t4, jb = ja + 1;
