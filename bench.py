@@ -61,32 +61,33 @@ def decode_bytes(L: int, w=W64) -> int:
             + S * hkv * d * 2 * 2 + hq * d * 2 + hq * d * 4 + hq * 4)
 
 
-def kernel_source_hash() -> str:
-    """sha256 (first 16 hex) of the kernel sources and the ABI header."""
-    import glob
+DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh")
+PREFILL_SOURCES = ("hga_common.cuh", "hga_tcgen05.cuh", "hga_prefill_attn.cuh")
+
+
+def kernel_source_hash(names=DECODE_SOURCES) -> str:
+    """sha256 (first 16 hex) of the device-code files one kernel is built from."""
     import hashlib
 
-    files = sorted(glob.glob(os.path.join(ROOT, "hierarchical_routed_sparse_build_b200", "csrc", "*")))
-    files.append(os.path.join(ROOT, "include", "hga.h"))
     h = hashlib.sha256()
-    for f in files:
-        with open(f, "rb") as fh:
+    for n in names:
+        with open(os.path.join(ROOT, "hierarchical_routed_sparse_build_b200", "csrc", n), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it covers these sources."""
+def profiled_traffic(profile="decode_64k_routed_kernel.md", names=DECODE_SOURCES):
+    """DRAM bytes per launch from a committed ncu summary, if it covers the current sources."""
     import re
 
-    path = os.path.join(ROOT, "profiles", "decode_64k_routed_kernel.md")
+    path = os.path.join(ROOT, "profiles", profile)
     try:
         text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(names):
         return None
     return int(m_bytes.group(1))
 
@@ -100,9 +101,13 @@ def bf16_peak():
         return 1590.0, 1400.0, "fallback"
 
 
-def prefill_flops(keys_per_block: int, w=synth.PREFILL_64K) -> int:
-    """QK^T and PV flops of a prefill: every (query, head) against its block's keys."""
-    return 2 * 2 * (w.n_new * w.n_q_heads) * keys_per_block * w.head_dim
+def prefill_flops(routed_total: int, n_pairs: int, w=synth.PREFILL_64K) -> int:
+    """Useful QK^T + PV flops of one prefill: every (query, head) against its routed keys and
+    its own causal prefix inside the block. routed_total = sum of routed counts over the
+    n_pairs (block, KV head) pairs."""
+    R = w.n_q_heads // w.n_kv_heads
+    keys = w.block * routed_total + n_pairs * (w.block * (w.block + 1) // 2)
+    return 4 * w.head_dim * R * keys
 
 
 def run_prefill(dev, steps: int, warmup: int):
@@ -156,21 +161,22 @@ def run_prefill(dev, steps: int, warmup: int):
     st, bits = hga.hga_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in prefill: {bits}")
-    keys = int(n_idx.sum().item()) // (nb * w.n_kv_heads) + w.block
-    fl = prefill_flops(keys)
+    fl = prefill_flops(int(n_idx.sum().item()), nb * w.n_kv_heads)
     burst, sustained, kind = bf16_peak()
     attn_tf = fl / (attend * 1e-3) / 1e12
     return {
         "workload": "prefill_2048_on_63488: 2048 new tokens in 32 blocks of 64 on a 63488-token cache, 32 q / "
                     "4 KV heads, d 128, block-shared routing (C 128, g 16, top-32 + sink + local, top-4 groups) "
-                    "+ own causal block; 2368 keys per block",
+                    "+ own causal block (2304 routed keys + the causal prefix of the block per query); flops count "
+                    "the useful QK^T and PV products",
         "tokens_per_s": round(T / (full * 1e-3), 1), "ms_per_step": round(full, 4),
         "route_ms": round(route, 4), "attend_ms": round(attend, 4),
         "flops_per_step": fl, "tflops_step": round(fl / (full * 1e-3) / 1e12, 1),
         "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel (tcgen05, TMEM accumulators)",
                      "achieved": round(attn_tf, 1), "peak": burst, "peak_kind": f"{kind} bf16 burst",
                      "unit": "TFLOP/s", "frac": round(attn_tf / burst, 4),
-                     "frac_of_sustained": round(attn_tf / sustained, 4)},
+                     "frac_of_sustained": round(attn_tf / sustained, 4),
+                     "traffic": profiled_traffic("prefill_64k_attn_kernel.md", PREFILL_SOURCES)},
     }
 
 
@@ -442,9 +448,15 @@ def main():
     ap.add_argument("--traffic", type=float, default=None, help="ncu dram bytes per launch, if measured")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the prefill workload (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.prefill_only:
+        import torch
+
+        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), args.steps, args.warmup)}), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
