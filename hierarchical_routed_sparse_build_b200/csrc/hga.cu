@@ -14,6 +14,7 @@
 
 #include "hga.h"
 #include "hga_common.cuh"
+#include "hga_decode.cuh"
 #include "hga_prefill_attn.cuh"
 #include "hga_prefill_route.cuh"
 #include "hga_routed.cuh"
@@ -23,6 +24,7 @@ namespace hga {
 namespace {
 
 std::atomic<int> g_ctas_per_head{0};
+std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 phase-by-phase, 2 fused
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -183,6 +185,49 @@ hga_status run_routed(RoutedArgs a, int D, int units, cudaStream_t stream) {
   const int P = pick_cluster(units);
   cudaError_t e = D == 128 ? launch_routed<128, MODE>(a, units, P, stream)
                            : launch_routed<64, MODE>(a, units, P, stream);
+  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+template <int D>
+cudaError_t launch_decode(const RoutedArgs& a, int units, int P, cudaStream_t stream) {
+  const DecodeSmem lay(D, a.n_pad, a.kcap, a.C / a.g);
+  auto kern = decode_kernel<D>;
+  static std::atomic<int> smem_set[kMaxDevices];
+  static std::atomic<bool> np_set[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (lay.total > smem_set[dev].load()) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    if (e != cudaSuccess) return e;
+    smem_set[dev].store(lay.total);
+  }
+  if (P > 8 && !np_set[dev].load()) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    np_set[dev].store(true);
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3((unsigned)(units * P), 1, 1);
+  cfg.blockDim = dim3(kRoutedThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)lay.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+hga_status run_decode(RoutedArgs a, int D, int units, cudaStream_t stream) {
+  if (DecodeSmem(D, a.n_pad, a.kcap, a.C / a.g).total > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
+  const int P = pick_cluster(units);
+  cudaError_t e = D == 128 ? launch_decode<128>(a, units, P, stream) : launch_decode<64>(a, units, P, stream);
   return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
 }
 
@@ -474,6 +519,8 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
   a.idx_out = idx;
   a.n_idx_out = n_idx;
   a.idx_stride = idx ? idx_stride : 0;
+  if (g_decode_kernel.load() != 1 && p->group % 16 == 0)
+    return run_decode(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
   return run_routed<kModeDecode>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
 }
 
@@ -563,6 +610,11 @@ hga_status hga_set_launch_option(int32_t option, int32_t value) {
   if (option == HGA_OPT_CTAS_PER_HEAD) {
     if (value < 0 || value > 16) return HGA_ERR_INVALID_ARG;
     g_ctas_per_head.store(value);
+    return HGA_OK;
+  }
+  if (option == HGA_OPT_DECODE_KERNEL) {
+    if (value < 0 || value > 2) return HGA_ERR_INVALID_ARG;
+    g_decode_kernel.store(value);
     return HGA_OK;
   }
   return HGA_ERR_INVALID_ARG;

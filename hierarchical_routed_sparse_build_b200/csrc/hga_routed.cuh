@@ -299,6 +299,97 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
     if (keys[i] >= kth) sel[pos++] = (int)route_key_id(keys[i]);
 }
 
+// Per-warp softmax states -> CTA partial (shared memory) -> output. A single-CTA
+// cluster writes out/lse directly; otherwise the CTAs combine their partials
+// through DSMEM, CTA cr finalising heads cr, cr + P, ... Every thread of every
+// CTA of the cluster must call it.
+template <int D>
+__device__ __forceinline__ void finish_attention(AttnState<D>& st, const RoutedArgs& a, cg::cluster_group& cluster,
+                                                 int P, int cr, int b, int h, float* red_o, float* red_m,
+                                                 float* red_l, float* cta_o, float* cta_m, float* cta_l) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __syncthreads();  // every warp is done with its tile before red_o reuses the region
+
+  // warp partials -> shared memory
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    st.l0 += __shfl_xor_sync(0xFFFFFFFFu, st.l0, off);
+    st.l1 += __shfl_xor_sync(0xFFFFFFFFu, st.l1, off);
+  }
+  {
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int h0 = 2 * t4, h1 = 2 * t4 + 1;
+    float* wo = red_o + warp * kMaxHeadsPerKv * D;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const int d0 = o_row(mt, g8);
+      wo[h0 * D + d0] = st.o[mt][0];
+      wo[h1 * D + d0] = st.o[mt][1];
+      wo[h0 * D + d0 + 1] = st.o[mt][2];
+      wo[h1 * D + d0 + 1] = st.o[mt][3];
+    }
+    if (g8 == 0) {
+      red_m[warp * kMaxHeadsPerKv + h0] = st.m0;
+      red_m[warp * kMaxHeadsPerKv + h1] = st.m1;
+      red_l[warp * kMaxHeadsPerKv + h0] = st.l0;
+      red_l[warp * kMaxHeadsPerKv + h1] = st.l1;
+    }
+  }
+  __syncthreads();
+  // CTA combine over warps; a single-CTA cluster writes the output directly.
+  for (int i = tid; i < a.R * D; i += kRoutedThreads) {
+    const int n = i / D, dd = i - n * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kRoutedWarps; ++w) M = fmaxf(M, red_m[w * kMaxHeadsPerKv + n]);
+    float acc = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kRoutedWarps; ++w) {
+        const float f = ex2(red_m[w * kMaxHeadsPerKv + n] - M);  // -inf -> 0
+        acc = fmaf(red_o[(w * kMaxHeadsPerKv + n) * D + dd], f, acc);
+        den = fmaf(red_l[w * kMaxHeadsPerKv + n], f, den);
+      }
+    }
+    if (P == 1) {
+      const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
+      a.out[head * D + dd] = den > 0.f ? acc / den : 0.f;
+      if (dd == 0 && a.lse != nullptr)
+        a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
+    } else {
+      cta_o[n * D + dd] = acc;
+      if (dd == 0) {
+        cta_m[n] = M;
+        cta_l[n] = den;
+      }
+    }
+  }
+  if (P > 1) {
+    cluster.sync();
+    // cluster combine: CTA cr finalises heads cr, cr + P, ... (all (head, d)
+    // pairs of this CTA in parallel)
+    const int my_heads = cr < a.R ? (a.R - cr + P - 1) / P : 0;
+    for (int i = tid; i < my_heads * D; i += kRoutedThreads) {
+      const int n = cr + P * (i / D), dd = i % D;
+      float M = -INFINITY;
+      for (int pr = 0; pr < P; ++pr) M = fmaxf(M, cluster.map_shared_rank(cta_m, pr)[n]);
+      float acc = 0.f, den = 0.f;
+      if (M != -INFINITY) {
+        for (int pr = 0; pr < P; ++pr) {
+          const float f = ex2(cluster.map_shared_rank(cta_m, pr)[n] - M);  // -inf -> 0
+          acc = fmaf(cluster.map_shared_rank(cta_o, pr)[n * D + dd], f, acc);
+          den = fmaf(cluster.map_shared_rank(cta_l, pr)[n], f, den);
+        }
+      }
+      const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
+      a.out[head * D + dd] = den > 0.f ? acc / den : 0.f;
+      if (dd == 0 && a.lse != nullptr)
+        a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
+    }
+    cluster.sync();
+  }
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -527,86 +618,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) routed_kernel(const RoutedA
       __syncthreads();
       attend_tiles<D>(st, rows, n_e, warp, kRoutedWarps, Kp, Vp, qfrag, tile, a.scale_log2, lane);
     }
-    __syncthreads();  // every warp is done with its tile before red_o reuses the region
-
-    // warp partials -> shared memory
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      st.l0 += __shfl_xor_sync(0xFFFFFFFFu, st.l0, off);
-      st.l1 += __shfl_xor_sync(0xFFFFFFFFu, st.l1, off);
-    }
-    {
-      const int g8 = lane >> 2, t4 = lane & 3;
-      const int h0 = 2 * t4, h1 = 2 * t4 + 1;
-      float* wo = red_o + warp * kMaxHeadsPerKv * D;
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        const int d0 = o_row(mt, g8);
-        wo[h0 * D + d0] = st.o[mt][0];
-        wo[h1 * D + d0] = st.o[mt][1];
-        wo[h0 * D + d0 + 1] = st.o[mt][2];
-        wo[h1 * D + d0 + 1] = st.o[mt][3];
-      }
-      if (g8 == 0) {
-        red_m[warp * kMaxHeadsPerKv + h0] = st.m0;
-        red_m[warp * kMaxHeadsPerKv + h1] = st.m1;
-        red_l[warp * kMaxHeadsPerKv + h0] = st.l0;
-        red_l[warp * kMaxHeadsPerKv + h1] = st.l1;
-      }
-    }
-    __syncthreads();
-    // CTA combine over warps; a single-CTA cluster writes the output directly.
-    for (int i = tid; i < a.R * D; i += kRoutedThreads) {
-      const int n = i / D, dd = i - n * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kRoutedWarps; ++w) M = fmaxf(M, red_m[w * kMaxHeadsPerKv + n]);
-      float acc = 0.f, den = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kRoutedWarps; ++w) {
-          const float f = ex2(red_m[w * kMaxHeadsPerKv + n] - M);  // -inf -> 0
-          acc = fmaf(red_o[(w * kMaxHeadsPerKv + n) * D + dd], f, acc);
-          den = fmaf(red_l[w * kMaxHeadsPerKv + n], f, den);
-        }
-      }
-      if (P == 1) {
-        const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
-        a.out[head * D + dd] = den > 0.f ? acc / den : 0.f;
-        if (dd == 0 && a.lse != nullptr)
-          a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
-      } else {
-        cta_o[n * D + dd] = acc;
-        if (dd == 0) {
-          cta_m[n] = M;
-          cta_l[n] = den;
-        }
-      }
-    }
-    if (P > 1) {
-      cluster.sync();
-      // cluster combine: CTA cr finalises heads cr, cr + P, ... (all (head, d)
-      // pairs of this CTA in parallel)
-      const int my_heads = cr < a.R ? (a.R - cr + P - 1) / P : 0;
-      for (int i = tid; i < my_heads * D; i += kRoutedThreads) {
-        const int n = cr + P * (i / D), dd = i % D;
-        float M = -INFINITY;
-        for (int pr = 0; pr < P; ++pr) M = fmaxf(M, cluster.map_shared_rank(cta_m, pr)[n]);
-        float acc = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-          for (int pr = 0; pr < P; ++pr) {
-            const float f = ex2(cluster.map_shared_rank(cta_m, pr)[n] - M);  // -inf -> 0
-            acc = fmaf(cluster.map_shared_rank(cta_o, pr)[n * D + dd], f, acc);
-            den = fmaf(cluster.map_shared_rank(cta_l, pr)[n], f, den);
-          }
-        }
-        const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
-        a.out[head * D + dd] = den > 0.f ? acc / den : 0.f;
-        if (dd == 0 && a.lse != nullptr)
-          a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
-      }
-      cluster.sync();
-    }
+    finish_attention<D>(st, a, cluster, P, cr, b, h, red_o, red_m, red_l, cta_o, cta_m, cta_l);
   }
 }
 

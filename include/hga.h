@@ -256,9 +256,14 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
  *   HGA_OPT_CTAS_PER_HEAD: CTAs (one thread-block cluster) that cooperate on one
  *   (sequence, KV head) in hga_route / hga_attend / hga_decode; 0 = automatic,
  *   1..16 otherwise (above 8 needs non-portable cluster support).
+ *   HGA_OPT_DECODE_KERNEL: which kernel runs hga_decode. 0 = automatic (the
+ *   fused kernel that routes groups inside the attention warps when group % 16
+ *   == 0, else the phase-by-phase kernel), 1 = always the phase-by-phase kernel
+ *   (the one hga_route and hga_attend use), 2 = the fused kernel where it
+ *   applies. Both compute the same routed set and attention.
  * Returns HGA_ERR_INVALID_ARG for an unknown option or value.
  */
-enum { HGA_OPT_CTAS_PER_HEAD = 1 };
+enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2 };
 hga_status hga_set_launch_option(int32_t option, int32_t value);
 
 /*

@@ -59,7 +59,8 @@ def run_and_check(hga, w, inp, units=None, check_summaries=True):
     B = len(inp.seq_lens)
     units = units or [(b, h) for b in range(B) for h in range(w.n_kv_heads)]
     idx_h, n_h = idx.cpu().numpy(), n_idx.cpu().numpy()
-    assert np.array_equal(idx_d.cpu().numpy(), idx_h) and np.array_equal(n_idx_d.cpu().numpy(), n_h)
+    idx_dh, n_dh = idx_d.cpu().numpy(), n_idx_d.cpu().numpy()
+    assert np.array_equal(n_dh, n_h)
     out_h, lse_h = out_d.cpu().numpy(), lse_d.cpu().numpy()
     cs_gpu, gs_gpu = bits(c.chunk_sum), bits(c.group_sum)
     # attention on the oracle's own token lists
@@ -89,9 +90,17 @@ def run_and_check(hga, w, inp, units=None, check_summaries=True):
         sl = slice(h * R, (h + 1) * R)
         assert_attention_close(out_a[b, sl], ref["out"], f"attend b{b} h{h}")
         assert_lse_close(lse_a[b, sl], ref["lse"], f"attend lse b{b} h{h}")
-        if same:
-            assert_attention_close(out_h[b, sl], ref["out"], f"decode b{b} h{h}")
-            assert_lse_close(lse_h[b, sl], ref["lse"], f"decode lse b{b} h{h}")
+        # the fused decode routes on its own (fp32 scores summed in another order
+        # than hga_route): its list must pass the same check, and its attention
+        # must match the oracle's attention over that list
+        toks_d = idx_dh[b, h, :n_dh[b, h]]
+        if not np.array_equal(toks_d, toks):
+            check_route(toks_d, ref["q"], ref["cs"], ref["gs"], L, w.chunk, w.group, w.top_chunks, w.top_groups,
+                        f"decode route b{b} h{h}")
+        ref_d, lse_ref_d = (ref["out"], ref["lse"]) if np.array_equal(toks_d, ref["tok"]) else \
+            oracle.attend(ref["q"], ref["K"], ref["V"], toks_d.astype(np.int64), with_lse=True)
+        assert_attention_close(out_h[b, sl], ref_d, f"decode b{b} h{h}")
+        assert_lse_close(lse_h[b, sl], lse_ref_d, f"decode lse b{b} h{h}")
     return exact, len(refs)
 
 
@@ -156,16 +165,33 @@ def test_full_coverage_is_dense_attention(hga):
             assert_attention_close(out[b, h * 8:(h + 1) * 8].cpu().numpy(), ref, f"dense b{b} h{h}")
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
 @pytest.mark.parametrize("ctas", [1, 2, 3, 8, 16])
-def test_cluster_sizes_agree(hga, ctas):
+def test_cluster_sizes_agree(hga, ctas, kernel):
     w = synth.with_len(synth.DECODE_64K, 16384)
     inp = synth.decode_inputs(w)
     hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, ctas)
+    hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, kernel)
     try:
         exact, n = run_and_check(hga, w, inp, check_summaries=False)
     finally:
         hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
+        hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, 0)
     assert exact >= n - 1
+
+
+@pytest.mark.parametrize("group,chunk,top_groups", [(8, 128, 4), (32, 128, 2), (16, 64, 4), (16, 256, 3)])
+def test_group_sizes(hga, group, chunk, top_groups):
+    # g = 8 runs the phase-by-phase kernel (a 16-token tile spans two groups);
+    # g = 32 and chunk 256 run the fused kernel with two tiles per group and 16
+    # groups per chunk; top_groups = C/g (all groups) runs its whole-chunk path
+    w = synth.Workload(f"g{group}c{chunk}", 1, 32, 4, 128, 6000, chunk, group, 5, top_groups, -1, 23)
+    inp = synth.decode_inputs(w, lengths=[6000, 4099, 777], max_len=6016)
+    exact, n = run_and_check(hga, w, inp)
+    assert exact >= n - 1
+    w_all = synth.Workload(f"g{group}c{chunk}all", 1, 32, 4, 128, 6000, chunk, group, 5, chunk // group, -1, 29)
+    inp = synth.decode_inputs(w_all, lengths=[6000, 2222], max_len=6016)
+    run_and_check(hga, w_all, inp)
 
 
 def test_attend_arbitrary_token_order_and_ragged_list(hga):
