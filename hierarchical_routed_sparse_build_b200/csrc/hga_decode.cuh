@@ -18,7 +18,8 @@
 //       across lanes with a halving butterfly (one score per lane pair). The
 //       64-bit keys (score bits, then lower id) go to every CTA of the cluster.
 //   --  cluster barrier
-//   R2  every CTA selects the top-k chunk ids (bucket select, ascending ids).
+//   R2  every CTA selects the top-k chunk ids (bucket select, ascending ids);
+//       warps whose first tile is always kept have its K/V loads in flight.
 //   A   the (CTA, warp) slots s = warp * P + cr take kept chunks s, s + P*W, ...
 //       and a share of the always-kept tiles (sink chunk, local chunk + tail),
 //       the shares balancing the tile counts. A warp first runs its always-kept
@@ -52,9 +53,9 @@ struct DecodeSmem {
     pages = o;   o = up16(o + 4 * (n_pad + 4));
     red_m = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
     red_l = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
-    cta_o = o;   o = up16(o + 4 * kMaxHeadsPerKv * D);
-    cta_m = o;   o = up16(o + 4 * kMaxHeadsPerKv);
-    cta_l = o;   o = up16(o + 4 * kMaxHeadsPerKv);
+    cta_o = o;   o = up16(o + 4 * kGatherSlots * D);
+    cta_m = o;   o = up16(o + 4 * kGatherSlots);
+    cta_l = o;   o = up16(o + 4 * kGatherSlots);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
     hist = o;    o = up16(o + 4 * kBuckets);
     misc = o;    o = up16(o + 4 * 32);
@@ -159,12 +160,6 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) decode_kernel(const RoutedA
   // Peers write keys into this CTA's shared memory in R1: every CTA of the
   // cluster must have started first (arrive now, wait before the first store).
   cluster_arrive_relaxed();
-  for (int e = tid; e < D; e += kRoutedThreads) {
-    float s = 0.f;
-    for (int i = 0; i < a.R; ++i) s += bf16_to_f(qb[(int64_t)i * D + e]);
-    qsum[e] = s;
-  }
-  stage_q_fragments<D>(qfrag, qb, a.R, tid, kRoutedThreads);
   if (paged) {
     // physical page of every page slot the context touches (page = chunk)
     const int n_slots = (L + C - 1) / C;
@@ -176,45 +171,54 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) decode_kernel(const RoutedA
       }
       pages[i] = page;
     }
+    __syncthreads();
   }
+
+  // R1 setup; its first loads go out before the head-summed query is formed
+  const bool select_needed = n_cand > r;
+  const int c0 = (int)((int64_t)n_cand * cr / P), c1 = (int)((int64_t)n_cand * (cr + 1) / P);
+  const int n_rows = c1 - c0;
+  const int nb = select_needed ? (n_rows + 15) / 16 : 0;
+  float qv[8];
+  auto issue = [&](int bi, uint4(&x)[NLD]) {
+#pragma unroll
+    for (int k = 0; k < NLD; ++k) {
+      const int i = min(16 * bi + RPI * k + rsub, n_rows - 1);
+      const int c = c0 + i + 1;
+      x[k] = ldg_stream(a.sv.chunk + a.sv.chunk_off(paged, b, h, hkv, c, paged ? pages[c] : 0) + 8 * u);
+    }
+  };
+  auto consume = [&](int bi, const uint4(&x)[NLD]) {
+    float v[NLD];
+#pragma unroll
+    for (int k = 0; k < NLD; ++k) v[k] = dot8(x[k], qv);
+    int idx;
+    const float score = butterfly_sum<NLD>(v, lane, idx);
+    const int i = 16 * bi + RPI * idx + rsub;
+    if ((lane & 1) == 0 && i < n_rows) {
+      const int cand = c0 + i;
+      const uint64_t key = route_key(score, (uint32_t)(cand + 1));
+      for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(keys, pr)[cand] = key;
+    }
+  };
+  uint4 xa[NLD], xb[NLD];
+  if (warp < nb) issue(warp, xa);
+  if (warp + kRoutedWarps < nb) issue(warp + kRoutedWarps, xb);
+
+  for (int e = tid; e < D; e += kRoutedThreads) {
+    float sq = 0.f;
+    for (int i = 0; i < a.R; ++i) sq += bf16_to_f(qb[(int64_t)i * D + e]);
+    qsum[e] = sq;
+  }
+  stage_q_fragments<D>(qfrag, qb, a.R, tid, kRoutedThreads);
   __syncthreads();
   cluster_wait();
 
   // ------------------------------------------------------------------ R1
-  const bool select_needed = n_cand > r;
-  if (select_needed) {
-    const int c0 = (int)((int64_t)n_cand * cr / P), c1 = (int)((int64_t)n_cand * (cr + 1) / P);
-    const int n_rows = c1 - c0;
-    const int nb = (n_rows + 15) / 16;
-    float qv[8];
+  if (nb > 0) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) qv[j] = qsum[8 * u + j];
-    auto issue = [&](int bi, uint4(&x)[NLD]) {
-#pragma unroll
-      for (int k = 0; k < NLD; ++k) {
-        const int i = min(16 * bi + RPI * k + rsub, n_rows - 1);
-        const int c = c0 + i + 1;
-        x[k] = ldg_stream(a.sv.chunk + a.sv.chunk_off(paged, b, h, hkv, c, paged ? pages[c] : 0) + 8 * u);
-      }
-    };
-    auto consume = [&](int bi, const uint4(&x)[NLD]) {
-      float v[NLD];
-#pragma unroll
-      for (int k = 0; k < NLD; ++k) v[k] = dot8(x[k], qv);
-      int idx;
-      const float score = butterfly_sum<NLD>(v, lane, idx);
-      const int i = 16 * bi + RPI * idx + rsub;
-      if ((lane & 1) == 0 && i < n_rows) {
-        const int cand = c0 + i;
-        const uint64_t key = route_key(score, (uint32_t)(cand + 1));
-        for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(keys, pr)[cand] = key;
-      }
-    };
-    uint4 xa[NLD], xb[NLD];
-    int bi = warp;
-    if (bi < nb) issue(bi, xa);
-    if (bi + kRoutedWarps < nb) issue(bi + kRoutedWarps, xb);
-    for (; bi < nb; bi += 2 * kRoutedWarps) {
+    for (int bi = warp; bi < nb; bi += 2 * kRoutedWarps) {
       consume(bi, xa);
       if (bi + 2 * kRoutedWarps < nb) issue(bi + 2 * kRoutedWarps, xa);
       if (bi + kRoutedWarps < nb) {
@@ -225,15 +229,8 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) decode_kernel(const RoutedA
   }
   cluster.sync();
 
-  // ------------------------------------------------------------------ R2
-  if (select_needed) {
-    select_top_chunks(keys, n_cand, r, sel, hist, misc, scratch, kDecodeScratchKeys);
-  } else {
-    for (int i = tid; i < r; i += kRoutedThreads) sel[i] = i + 1;
-  }
-  __syncthreads();
-
   // ------------------------------------------------------------------- A
+  // (set up before the select, which only the routed-chunk tiles depend on)
   const bool all_groups = gk >= gpc;
   const int gsel = all_groups ? gpc : gk;  // groups kept per routed chunk
   const int gt = g / 16;                   // tiles per group
@@ -244,6 +241,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) decode_kernel(const RoutedA
   const int S = dense ? L : C + r * span + (L - tail0);
   const int NS = kRoutedWarps * P;
   const int s = warp * P + cr;
+  // routed chunk i goes to slot i % NS; this slot's chunks are s, s + NS, ...
   const int n_mine = s < r ? (r - s + NS - 1) / NS : 0;
   // always-kept tiles of this slot: [fa0, fa1) tops up slots that hold one
   // routed chunk fewer (s >= r % NS), the rest [fb0, fb1) is spread evenly
@@ -371,14 +369,34 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) decode_kernel(const RoutedA
 
   AttnState<D> st;
   st.init();
-  if (n_mine > 0 && !all_groups) issue_groups(0);
-  if (n_tiles > 0) {
-    const uint16_t* Kp = a.kv.k;
-    const uint16_t* Vp = a.kv.v;
-    TileRef cur = tile_at(0);
-    uint4 kr[NLD], vr[NLD];
+  const uint16_t* Kp = a.kv.k;
+  const uint16_t* Vp = a.kv.v;
+  uint4 kr[NLD], vr[NLD];
+  TileRef cur;
+  cur.row0 = 0;
+  cur.nvalid = 0;
+  // a warp whose first tile is always kept loads it under the chunk select
+  if (nF > 0) {
+    cur = tile_at(0);
     fetch(kr, Kp, cur);
     fetch(vr, Vp, cur);
+  }
+
+  // ------------------------------------------------------------------ R2
+  if (select_needed) {
+    select_top_chunks(keys, n_cand, r, sel, hist, misc, scratch, kDecodeScratchKeys);
+  } else {
+    for (int i = tid; i < r; i += kRoutedThreads) sel[i] = i + 1;
+  }
+  __syncthreads();
+
+  if (n_mine > 0 && !all_groups) issue_groups(0);
+  if (n_tiles > 0) {
+    if (nF == 0) {
+      cur = tile_at(0);
+      fetch(kr, Kp, cur);
+      fetch(vr, Vp, cur);
+    }
     for (int q = 0; q < n_tiles; ++q) {
       const bool more = q + 1 < n_tiles;
       TileRef nx = cur;

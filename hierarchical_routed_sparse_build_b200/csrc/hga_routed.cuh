@@ -48,6 +48,9 @@ constexpr int kBuckets = 1024;             // bucket-select histogram size
 // max, [24..31] per-warp scan totals
 static_assert(kRoutedWarps <= 8, "misc[] holds at most 8 per-warp slots");
 constexpr int kStageBytes = 32 * 1024;     // routing: double-buffered summary staging
+// Cluster combine: CTA n % P finalises head n and receives P * ceil(R / P)
+// partials, at most 16 for R <= 8 and P <= 16.
+constexpr int kGatherSlots = 16;
 
 struct RoutedArgs {
   KvView kv;
@@ -83,9 +86,9 @@ struct RoutedSmem {
     rows = o;    o = up16(o + 4 * kEntryBatch);
     red_m = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
     red_l = o;   o = up16(o + 4 * kRoutedWarps * kMaxHeadsPerKv);
-    cta_o = o;   o = up16(o + 4 * kMaxHeadsPerKv * D);
-    cta_m = o;   o = up16(o + 4 * kMaxHeadsPerKv);
-    cta_l = o;   o = up16(o + 4 * kMaxHeadsPerKv);
+    cta_o = o;   o = up16(o + 4 * kGatherSlots * D);
+    cta_m = o;   o = up16(o + 4 * kGatherSlots);
+    cta_l = o;   o = up16(o + 4 * kGatherSlots);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
     hist = o;    o = up16(o + 4 * kBuckets);
     misc = o;    o = up16(o + 4 * 32);
@@ -296,7 +299,7 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
   for (int i = s0; i < s1; ++i) cnt += keys[i] >= kth;
   int pos = block_exclusive_scan(cnt, misc + 24);
   for (int i = s0; i < s1; ++i)
-    if (keys[i] >= kth) sel[pos++] = (int)route_key_id(keys[i]);
+    if (keys[i] >= kth && pos < r) sel[pos++] = (int)route_key_id(keys[i]);
 }
 
 // Per-warp softmax states -> CTA partial (shared memory) -> output. A single-CTA
@@ -336,7 +339,11 @@ __device__ __forceinline__ void finish_attention(AttnState<D>& st, const RoutedA
     }
   }
   __syncthreads();
-  // CTA combine over warps; a single-CTA cluster writes the output directly.
+  // CTA combine over warps. A single-CTA cluster writes the output directly;
+  // otherwise head n is finalised by CTA n % P, and every CTA pushes its
+  // partial of head n into that CTA's gather slot cr * HPC + n / P (remote
+  // stores, then one cluster barrier; the finalising reads are local).
+  const int HPC = (a.R + P - 1) / P;
   for (int i = tid; i < a.R * D; i += kRoutedThreads) {
     const int n = i / D, dd = i - n * D;
     float M = -INFINITY;
@@ -357,28 +364,29 @@ __device__ __forceinline__ void finish_attention(AttnState<D>& st, const RoutedA
       if (dd == 0 && a.lse != nullptr)
         a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
     } else {
-      cta_o[n * D + dd] = acc;
+      const int owner = n % P, slot = cr * HPC + n / P;
+      cluster.map_shared_rank(cta_o, owner)[slot * D + dd] = acc;
       if (dd == 0) {
-        cta_m[n] = M;
-        cta_l[n] = den;
+        cluster.map_shared_rank(cta_m, owner)[slot] = M;
+        cluster.map_shared_rank(cta_l, owner)[slot] = den;
       }
     }
   }
   if (P > 1) {
+    // After this barrier no CTA touches another's shared memory, so there is
+    // no closing barrier.
     cluster.sync();
-    // cluster combine: CTA cr finalises heads cr, cr + P, ... (all (head, d)
-    // pairs of this CTA in parallel)
     const int my_heads = cr < a.R ? (a.R - cr + P - 1) / P : 0;
     for (int i = tid; i < my_heads * D; i += kRoutedThreads) {
-      const int n = cr + P * (i / D), dd = i % D;
+      const int jj = i / D, dd = i - jj * D, n = cr + P * jj;
       float M = -INFINITY;
-      for (int pr = 0; pr < P; ++pr) M = fmaxf(M, cluster.map_shared_rank(cta_m, pr)[n]);
+      for (int pr = 0; pr < P; ++pr) M = fmaxf(M, cta_m[pr * HPC + jj]);
       float acc = 0.f, den = 0.f;
       if (M != -INFINITY) {
         for (int pr = 0; pr < P; ++pr) {
-          const float f = ex2(cluster.map_shared_rank(cta_m, pr)[n] - M);  // -inf -> 0
-          acc = fmaf(cluster.map_shared_rank(cta_o, pr)[n * D + dd], f, acc);
-          den = fmaf(cluster.map_shared_rank(cta_l, pr)[n], f, den);
+          const float f = ex2(cta_m[pr * HPC + jj] - M);  // -inf -> 0
+          acc = fmaf(cta_o[(pr * HPC + jj) * D + dd], f, acc);
+          den = fmaf(cta_l[pr * HPC + jj], f, den);
         }
       }
       const int64_t head = (int64_t)b * a.hq + (int64_t)h * a.R + n;
@@ -386,7 +394,6 @@ __device__ __forceinline__ void finish_attention(AttnState<D>& st, const RoutedA
       if (dd == 0 && a.lse != nullptr)
         a.lse[head] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994530942f : -INFINITY;
     }
-    cluster.sync();
   }
 }
 
