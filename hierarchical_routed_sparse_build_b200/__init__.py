@@ -24,7 +24,8 @@ __all__ = [
     "hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
-    "hga_prefill", "hga_prefill_noalloc", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL", "STATUS_NAMES",
+    "hga_prefill", "hga_prefill_noalloc", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
+    "HGA_OPT_PREFILL_KERNEL", "STATUS_NAMES",
     "EXPORTED",
 ]
 
@@ -34,6 +35,7 @@ _LIB_PATH = os.path.join(_HERE, "libhga.so")
 HGA_OK = 0
 HGA_OPT_CTAS_PER_HEAD = 1
 HGA_OPT_DECODE_KERNEL = 2
+HGA_OPT_PREFILL_KERNEL = 3
 STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_UNSUPPORTED", 3: "HGA_ERR_CUDA",
                 4: "HGA_ERR_DEVICE_FAULT", 5: "HGA_ERR_TIMEOUT"}
 EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",

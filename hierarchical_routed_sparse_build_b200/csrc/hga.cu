@@ -16,6 +16,7 @@
 #include "hga_common.cuh"
 #include "hga_decode.cuh"
 #include "hga_prefill_attn.cuh"
+#include "hga_prefill_attn2.cuh"
 #include "hga_prefill_route.cuh"
 #include "hga_routed.cuh"
 #include "hga_summaries.cuh"
@@ -25,6 +26,7 @@ namespace {
 
 std::atomic<int> g_ctas_per_head{0};
 std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 phase-by-phase, 2 fused
+std::atomic<int> g_prefill_kernel{0};  // 0 automatic (one Q tile per CTA), 1 one tile, 2 two tiles
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -349,6 +351,18 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
     configured[dev].store(true);
   }
   const int m_tiles = a.R * block / kPfRows;
+  if (m_tiles % 2 == 0 && g_prefill_kernel.load() == 2) {
+    static std::atomic<bool> configured2[kMaxDevices];
+    if (!configured2[dev].load()) {
+      if (cudaFuncSetAttribute(prefill_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Prefill2Smem::kTotal) != cudaSuccess)
+        return HGA_ERR_CUDA;
+      configured2[dev].store(true);
+    }
+    const int grid2 = (n_queries / block) * kv->n_kv_heads * (m_tiles / 2);
+    prefill_attn2_kernel<<<grid2, kPf2Threads, Prefill2Smem::kTotal, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+  }
   const int grid = (n_queries / block) * kv->n_kv_heads * m_tiles;
   prefill_attn_kernel<<<grid, kPfThreads, PrefillSmem::kTotal, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
@@ -615,6 +629,11 @@ hga_status hga_set_launch_option(int32_t option, int32_t value) {
   if (option == HGA_OPT_DECODE_KERNEL) {
     if (value < 0 || value > 2) return HGA_ERR_INVALID_ARG;
     g_decode_kernel.store(value);
+    return HGA_OK;
+  }
+  if (option == HGA_OPT_PREFILL_KERNEL) {
+    if (value < 0 || value > 2) return HGA_ERR_INVALID_ARG;
+    g_prefill_kernel.store(value);
     return HGA_OK;
   }
   return HGA_ERR_INVALID_ARG;

@@ -261,9 +261,15 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
  *   == 0, else the phase-by-phase kernel), 1 = always the phase-by-phase kernel
  *   (the one hga_route and hga_attend use), 2 = the fused kernel where it
  *   applies. Both compute the same routed set and attention.
+ *   HGA_OPT_PREFILL_KERNEL: which kernel runs the prefill attention. 0 =
+ *   automatic (currently the one-tile kernel, the faster of the two on the
+ *   2048-on-63488 workload), 1 = one 128-row query tile per CTA, 2 = two
+ *   tiles per CTA sharing each gathered key tile (warp-specialised, Q and P in
+ *   tensor memory) when the query heads per KV head are a multiple of 4, else
+ *   one tile. Both compute the same attention.
  * Returns HGA_ERR_INVALID_ARG for an unknown option or value.
  */
-enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2 };
+enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2, HGA_OPT_PREFILL_KERNEL = 3 };
 hga_status hga_set_launch_option(int32_t option, int32_t value);
 
 /*

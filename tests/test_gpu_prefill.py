@@ -21,6 +21,15 @@ def hga():
     return m
 
 
+@pytest.fixture(params=[1, 2], ids=["one_tile_per_cta", "two_tiles_per_cta"])
+def pf_kernel(hga, request):
+    """Run a test with each prefill attention kernel (two tiles per CTA needs R % 4 == 0;
+    otherwise the library uses the one-tile kernel either way)."""
+    hga.hga_set_launch_option(hga.HGA_OPT_PREFILL_KERNEL, request.param)
+    yield request.param
+    hga.hga_set_launch_option(hga.HGA_OPT_PREFILL_KERNEL, 0)
+
+
 def dev_bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
 
@@ -120,13 +129,13 @@ def small(hq, hkv, L0, T, k=8, G=2):
                           n_new=T, block=64)
 
 
-def test_prefill_small_aligned(hga):
+def test_prefill_small_aligned(hga, pf_kernel):
     w = small(32, 4, 4096, 256)
     exact, n = run_case(hga, w, 4096, 256)
     assert exact >= n - 1
 
 
-def test_prefill_small_ragged_cache(hga):
+def test_prefill_small_ragged_cache(hga, pf_kernel):
     # cache length not a multiple of the chunk or of 16: the local chunk carries a
     # tail and the block's own tokens start at an unaligned position
     w = small(16, 2, 5000 + 77, 192)
@@ -134,12 +143,12 @@ def test_prefill_small_ragged_cache(hga):
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 4), (16, 4), (8, 1)])
-def test_prefill_head_groups(hga, hq, hkv):
+def test_prefill_head_groups(hga, pf_kernel, hq, hkv):
     w = small(hq, hkv, 3000, 128)
     run_case(hga, w, 3000, 128)
 
 
-def test_prefill_dense_short_cache(hga):
+def test_prefill_dense_short_cache(hga, pf_kernel):
     # fewer than three full chunks in the cache: every cache token is attended
     w = small(8, 2, 300, 128)
     run_case(hga, w, 300, 128)
