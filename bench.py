@@ -285,6 +285,25 @@ def oracle_queries_per_s(inp, w, seconds: float, max_threads: int | None = None)
                                   f"({queries:.0f} queries) in {dt:.1f} s, summaries prebuilt"
 
 
+# --------------------------------------------------------------------------- ranks
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of x over all ranks (device time of the slowest rank); x itself for one process."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: units every rank processed in every step over the slowest rank's time."""
+    return units_per_rank * world * steps / (total_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 
@@ -347,14 +366,9 @@ def run_gpu(args, rank: int, world: int, dist):
     st, bits = hga.hga_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in timed region: {bits}")
-    total_ms = float(sum(times))
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(times)), dist, dev)
     ms_per_step = total_ms / args.steps
-    queries = B * world * args.steps
-    value = queries / (total_ms / 1e3)
+    value = weak_scaling_rate(B, world, args.steps, total_ms)
 
     # end to end through the public API with host buffers
     q_host = torch.from_numpy(inp.q.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -371,11 +385,7 @@ def run_gpu(args, rank: int, world: int, dist):
     for _ in range(3):
         e2e_step()
     e2e_times = timed(args.steps, e2e_step)
-    e2e_ms = float(sum(e2e_times))
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(float(sum(e2e_times)), dist, dev)
 
     # batch-1 latency and the context-length sweep (same kernels, same cache)
     sweep = {}
@@ -422,7 +432,7 @@ def run_gpu(args, rank: int, world: int, dist):
                      "traffic": args.traffic if args.traffic is not None else
                      (profiled_traffic() if B == 64 else None),
                      "alg_bytes_per_query": decode_bytes(w.ctx_len), "alg_bytes_per_launch": alg},
-        "e2e": {"value": round(B * world * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+        "e2e": {"value": round(weak_scaling_rate(B, world, args.steps, e2e_ms), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_host.numel() * 2),
                 "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4)},
         "clocks": clocks.summary(),
