@@ -61,7 +61,7 @@ def decode_bytes(L: int, w=W64) -> int:
             + S * hkv * d * 2 * 2 + hq * d * 2 + hq * d * 4 + hq * 4)
 
 
-DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh")
+DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh", "hga_decode.cuh")
 PREFILL_SOURCES = ("hga_common.cuh", "hga_tcgen05.cuh", "hga_prefill_attn.cuh")
 
 
@@ -76,7 +76,7 @@ def kernel_source_hash(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(profile="decode_64k_routed_kernel.md", names=DECODE_SOURCES):
+def profiled_traffic(profile="decode_64k_decode_kernel.md", names=DECODE_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, if it covers the current sources."""
     import re
 
@@ -426,7 +426,7 @@ def run_gpu(args, rank: int, world: int, dist):
                    "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
                    "l2": "flushed between steps (256 MiB read, outside the timed events)",
                    "ctas_per_head": args.ctas or "auto"},
-        "roofline": {"bound": "hbm", "kernel": "routed_kernel<128, decode> (whole step, one launch)",
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel<128> (fused routing + attention, one launch per step)",
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4),
                      "traffic": args.traffic if args.traffic is not None else
