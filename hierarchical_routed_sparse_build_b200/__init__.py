@@ -24,7 +24,8 @@ __all__ = [
     "hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
-    "hga_prefill", "hga_prefill_noalloc", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
+    "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
+    "hga_prefill_growing_workspace_size", "hga_prefill_growing", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
     "HGA_OPT_PREFILL_KERNEL", "STATUS_NAMES",
     "EXPORTED",
 ]
@@ -41,7 +42,8 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_UNSUPPORTED",
 EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",
             "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
             "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
-            "hga_prefill", "hga_prefill_noalloc")
+            "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
+            "hga_prefill_growing_workspace_size", "hga_prefill_growing")
 
 
 class HgaError(RuntimeError):
@@ -87,6 +89,10 @@ def _load() -> ctypes.CDLL:
         "hga_prefill_attend": ([vp, i32, i32, i32, KV, i32, vp, i32, vp, P, vp, vp], i32),
         "hga_prefill_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
         "hga_prefill": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
+        "hga_append": ([KV, vp, vp, vp, P, vp, vp, vp], i32),
+        "hga_route_blocks_growing": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, i32, vp, vp], i32),
+        "hga_prefill_growing_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
+        "hga_prefill_growing": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
         "hga_prefill_noalloc": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -217,6 +223,36 @@ def hga_prefill_noalloc(q, n_q_heads: int, n_queries: int, block: int, kv: hga_k
     _check(_lib.hga_prefill_noalloc(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
                                     _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(out),
                                     _stream(stream)), "hga_prefill_noalloc")
+
+
+def hga_append(kv: hga_kv, seq_lens, k_new, v_new, p: hga_params, chunk_sum, group_sum, stream=None) -> None:
+    """Append one token per sequence (k_new, v_new [B][Hkv][d] bf16) and refresh the completed chunk's
+    summaries; seq_lens (kv's length array) grows by one on the device."""
+    _check(_lib.hga_append(ctypes.byref(kv), _addr(seq_lens), _addr(k_new), _addr(v_new), ctypes.byref(p),
+                           _addr(chunk_sum), _addr(group_sum), _stream(stream)), "hga_append")
+
+
+def hga_route_blocks_growing(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int,
+                             chunk_sum, group_sum, p: hga_params, idx, idx_stride: int, n_idx, stream=None) -> None:
+    _check(_lib.hga_route_blocks_growing(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
+                                         _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(idx),
+                                         idx_stride, _addr(n_idx), _stream(stream)), "hga_route_blocks_growing")
+
+
+def hga_prefill_growing_workspace_size(kv: hga_kv, n_q_heads: int, n_queries: int, block: int, cache_len: int,
+                                       p: hga_params) -> int:
+    n = _lib.hga_prefill_growing_workspace_size(ctypes.byref(kv), n_q_heads, n_queries, block, cache_len,
+                                                ctypes.byref(p))
+    if n == 0:
+        raise HgaError(1, "hga_prefill_growing_workspace_size")
+    return n
+
+
+def hga_prefill_growing(q, n_q_heads: int, n_queries: int, block: int, kv: hga_kv, cache_len: int, chunk_sum,
+                        group_sum, p: hga_params, out, workspace, workspace_bytes: int, stream=None) -> None:
+    _check(_lib.hga_prefill_growing(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
+                                    _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(out),
+                                    _addr(workspace), workspace_bytes, _stream(stream)), "hga_prefill_growing")
 
 
 def hga_set_launch_option(option: int, value: int) -> None:

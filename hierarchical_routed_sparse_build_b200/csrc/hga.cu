@@ -278,7 +278,7 @@ hga_status check_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, in
 hga_status launch_block_route(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
                               const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
                               const hga_params* p, int32_t* idx, int32_t idx_stride, int32_t* n_idx,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, bool growing = false) {
   BlockRouteArgs a;
   std::memset(&a, 0, sizeof a);
   a.q = static_cast<const uint16_t*>(q);
@@ -298,6 +298,7 @@ hga_status launch_block_route(const void* q, int32_t n_q_heads, int32_t n_querie
   a.idx = idx;
   a.n_idx = n_idx;
   a.idx_stride = idx_stride;
+  a.growing = growing ? 1 : 0;
   const int n_pad = a.max_chunks - 2 > 2 ? a.max_chunks - 2 : 2;
   const int kcap_raw = a.max_chunks - 2 < a.k ? a.max_chunks - 2 : a.k;
   const int kcap = kcap_raw < 1 ? 1 : kcap_raw;
@@ -318,7 +319,8 @@ hga_status launch_block_route(const void* q, int32_t n_q_heads, int32_t n_querie
 
 hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
                                  const hga_kv* kv, int32_t cache_len, const int32_t* idx, int32_t idx_stride,
-                                 const int32_t* n_idx, const hga_params* p, float* out, cudaStream_t stream) {
+                                 const int32_t* n_idx, const hga_params* p, float* out, cudaStream_t stream,
+                                 bool growing = false) {
   PrefillAttnArgs a;
   std::memset(&a, 0, sizeof a);
   a.q = static_cast<const uint16_t*>(q);
@@ -336,6 +338,7 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
   a.idx_stride = idx_stride;
   a.scale_log2 = scale_log2(p, kv->head_dim);
   a.out = out;
+  a.growing = growing ? 1 : 0;
   static std::atomic<bool> configured[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
@@ -446,9 +449,38 @@ hga_status hga_build_summaries(const hga_kv* kv, const hga_params* p, void* chun
   dim3 block((unsigned)(32 * (gpc < 8 ? gpc : 8)));
   const size_t smem = (size_t)gpc * kv->head_dim * sizeof(float);
   if (kv->head_dim == 128)
-    summaries_kernel<128><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group);
+    summaries_kernel<128><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group, 0);
   else
-    summaries_kernel<64><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group);
+    summaries_kernel<64><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group, 0);
+  return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+hga_status hga_append(const hga_kv* kv, int32_t* seq_lens, const void* k_new, const void* v_new,
+                      const hga_params* p, void* chunk_sum, void* group_sum, cudaStream_t stream) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (seq_lens == nullptr || seq_lens != kv->seq_lens || k_new == nullptr || v_new == nullptr ||
+      !aligned16(k_new) || !aligned16(v_new) || chunk_sum == nullptr || group_sum == nullptr ||
+      !aligned16(chunk_sum) || !aligned16(group_sum))
+    return HGA_ERR_INVALID_ARG;
+  const KvView kvv = make_kv_view(kv);
+  const SumView sv = make_sum_view(kv, p, chunk_sum, group_sum);
+  uint16_t* k = static_cast<uint16_t*>(const_cast<void*>(kv->k));
+  uint16_t* v = static_cast<uint16_t*>(const_cast<void*>(kv->v));
+  const uint16_t* kn = static_cast<const uint16_t*>(k_new);
+  const uint16_t* vn = static_cast<const uint16_t*>(v_new);
+  const int gpc = p->chunk / p->group;
+  dim3 grid(1u, (unsigned)kv->n_kv_heads, (unsigned)kv->batch);
+  dim3 block((unsigned)(32 * (gpc < 8 ? gpc : 8)));
+  const size_t smem = (size_t)gpc * kv->head_dim * sizeof(float);
+  if (kv->head_dim == 128) {
+    append_kernel<128><<<kv->batch, 128, 0, stream>>>(kvv, k, v, seq_lens, kn, vn);
+    summaries_kernel<128><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group, 1);
+  } else {
+    append_kernel<64><<<kv->batch, 128, 0, stream>>>(kvv, k, v, seq_lens, kn, vn);
+    summaries_kernel<64><<<grid, block, smem, stream>>>(kvv, sv, p->chunk, p->group, 1);
+  }
   return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
 }
 
@@ -593,6 +625,66 @@ hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int3
                          n_idx, stream);
   if (s != HGA_OK) return s;
   return launch_prefill_attend(q, n_q_heads, n_queries, block, kv, cache_len, idx, stride, n_idx, p, out, stream);
+}
+
+// Routed count of the longest list over the blocks of a growing-history
+// prefill (block b routes over [0, cache_len + b * block)); the count is not
+// monotone in the length (the local chunk's tail shrinks at a chunk boundary).
+int routed_count_growing(int32_t cache_len, int32_t n_queries, int32_t block, const hga_params* p) {
+  int best = 0;
+  for (int b = 0; b * block < n_queries; ++b) {
+    const int c = routed_count(cache_len + b * block, p);
+    if (c > best) best = c;
+  }
+  return best;
+}
+
+hga_status hga_route_blocks_growing(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                    const hga_kv* kv, int32_t cache_len, const void* chunk_sum,
+                                    const void* group_sum, const hga_params* p, int32_t* idx, int32_t idx_stride,
+                                    int32_t* n_idx, cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, false);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+      idx == nullptr || n_idx == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if (idx_stride < routed_count_growing(cache_len, n_queries, block, p)) return HGA_ERR_INVALID_ARG;
+  return launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx,
+                            idx_stride, n_idx, stream, true);
+}
+
+size_t hga_prefill_growing_workspace_size(const hga_kv* kv, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                          int32_t cache_len, const hga_params* p) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK || block < 1 || n_queries < 1 ||
+      n_q_heads < 1 || cache_len < 0)
+    return 0;
+  const size_t units = (size_t)((n_queries + block - 1) / block) * kv->n_kv_heads;
+  const size_t stride = (size_t)routed_count_growing(cache_len, n_queries, block, p);
+  return units * (stride + 1) * sizeof(int32_t);
+}
+
+hga_status hga_prefill_growing(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                               const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                               const hga_params* p, float* out, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  hga_status s = check_prefill(q, n_q_heads, n_queries, block, kv, cache_len, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if (chunk_sum == nullptr || group_sum == nullptr || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+      out == nullptr || workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return HGA_ERR_INVALID_ARG;
+  const size_t need = hga_prefill_growing_workspace_size(kv, n_q_heads, n_queries, block, cache_len, p);
+  if (workspace_bytes < need) return HGA_ERR_INVALID_ARG;
+  const int stride = routed_count_growing(cache_len, n_queries, block, p);
+  const int units = (n_queries / block) * kv->n_kv_heads;
+  int32_t* idx = static_cast<int32_t*>(workspace);
+  int32_t* n_idx = idx + (size_t)units * stride;
+  s = launch_block_route(q, n_q_heads, n_queries, block, kv, cache_len, chunk_sum, group_sum, p, idx, stride,
+                         n_idx, stream, true);
+  if (s != HGA_OK) return s;
+  return launch_prefill_attend(q, n_q_heads, n_queries, block, kv, cache_len, idx, stride, n_idx, p, out, stream,
+                               true);
 }
 
 hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,

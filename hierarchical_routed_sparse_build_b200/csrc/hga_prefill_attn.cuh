@@ -40,6 +40,7 @@ struct PrefillAttnArgs {
   const uint16_t* v;
   int hkv, max_len;
   int cache_len;       // query i sits at position cache_len + i
+  int growing;         // nonzero: block b's routed tokens lie in [0, cache_len + b * block)
   const int32_t* idx;  // [n_blocks][Hkv][idx_stride] routed cache tokens
   const int32_t* n_idx;
   int idx_stride;
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
   const int qi = blk * a.block + p;
   const int64_t q_row = (int64_t)qi * a.hq + (int64_t)h * a.R + head_local;
   const int own0 = a.cache_len + blk * a.block;  // first own token of the block
+  const int hist = a.growing ? own0 : a.cache_len;  // routed tokens lie in [0, hist)
 
   int n_cache = __ldg(a.n_idx + unit);
   if (n_cache < 0 || n_cache > a.idx_stride) {
@@ -105,7 +107,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     return e < n_cache ? __ldg(ilist + e) : (e < n_keys ? own0 + (e - n_cache) : own0);
   };
   auto key_row = [&](int e, int tok) -> int64_t {
-    if (e < n_cache && (tok < 0 || tok >= a.cache_len)) {
+    if (e < n_cache && (tok < 0 || tok >= hist)) {
       report_error(kErrIndex);
       tok = own0;
     }

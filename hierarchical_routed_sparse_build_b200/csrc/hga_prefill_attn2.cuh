@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kPf2Threads, 1) prefill_attn2_kernel(const Pre
   const int n_keys = n_cache + a.block;
   const int n_tiles = (n_keys + kPfKeys - 1) / kPfKeys;
   const int own0 = a.cache_len + blk * a.block;  // first own token of the block
+  const int hist = a.growing ? own0 : a.cache_len;  // routed tokens lie in [0, hist)
 
   if (tid == 0) {
     for (int s = 0; s < kPf2Stages; ++s) {
@@ -241,7 +242,7 @@ __global__ void __launch_bounds__(kPf2Threads, 1) prefill_attn2_kernel(const Pre
       for (int k = 0; k < 4; ++k) {
         const int row = 8 * warp + 2 * k + ck;
         int tk = __shfl_sync(0xFFFFFFFFu, tok, 2 * k + ck);
-        if (jt * kPfKeys + row < n_cache && (tk < 0 || tk >= a.cache_len)) {
+        if (jt * kPfKeys + row < n_cache && (tk < 0 || tk >= hist)) {
           report_error(kErrIndex);
           tk = own0;
         }

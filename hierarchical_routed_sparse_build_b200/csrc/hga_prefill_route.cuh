@@ -28,6 +28,7 @@ struct BlockRouteArgs {
   const uint16_t* chunk_sum;  // [Hkv][max_chunks][D] (batch 1, contiguous)
   const uint16_t* group_sum;  // [Hkv][max_chunks][gpc][D]
   int hkv, max_chunks, L;     // L: cache length (routing covers [0, L))
+  int growing;                // nonzero: block b routes over [0, L + b * block) (its whole history)
   int C, g, k, G;
   int32_t* idx;    // [n_blocks][Hkv][idx_stride]
   int32_t* n_idx;  // [n_blocks][Hkv]
@@ -110,7 +111,8 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int W = kRoutedWarps;
   const int gpc = a.C / a.g, gk = a.G;
-  const int nf = a.L / a.C;
+  const int L = a.L + (a.growing ? blk * a.block : 0);  // routed history of this block
+  const int nf = L / a.C;
   const bool dense = nf <= 2;
   const int n_cand = dense ? 0 : nf - 2;
   const int r = n_cand < a.k ? n_cand : a.k;
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
     }
   }
   __syncthreads();
-  const int S = dense ? a.L : a.C + r * gk * a.g + (a.L - (nf - 1) * a.C);
+  const int S = dense ? L : a.C + r * gk * a.g + (L - (nf - 1) * a.C);
   const int unit = blk * a.hkv + h;
   const int span = gk * a.g;
   const int Sw = min(S, a.idx_stride);

@@ -16,11 +16,19 @@
 
 namespace hga {
 
+// last_only: the grid has one chunk column and each (head, sequence) CTA
+// summarises the chunk that the sequence's last token completed, if it did
+// (length a positive multiple of C); used after an append.
 template <int D>
-__global__ void __launch_bounds__(256) summaries_kernel(KvView kv, SumView sv, int C, int g) {
+__global__ void __launch_bounds__(256) summaries_kernel(KvView kv, SumView sv, int C, int g, int last_only) {
   extern __shared__ float group_acc[];  // [gpc][D]
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int L = kv.length(b);
+  int c = blockIdx.x;
+  if (last_only) {
+    if (L == 0 || L % C != 0) return;  // uniform over the CTA
+    c = L / C - 1;
+  }
   if (c >= L / C) return;  // uniform over the CTA
   const bool paged = kv.page_table != nullptr;
   int page = 0;
@@ -95,6 +103,33 @@ __global__ void __launch_bounds__(256) summaries_kernel(KvView kv, SumView sv, i
     float mean = c_pow2 ? s * inv_c : s / (float)C;
     sv.chunk[coff + e] = __bfloat16_as_ushort(__float2bfloat16_rn(mean));
   }
+}
+
+// Append one token to every sequence of the cache: K/V rows k_new[b][h],
+// v_new[b][h] go to position seq_lens[b] (a contiguous row, or the page slot
+// seq_lens[b] / page_size of a paged cache), then seq_lens[b] grows by one.
+// One CTA per sequence; the length is read before any thread writes it. A
+// length at max_len is reported (kErrSeqLen) and left unchanged.
+template <int D>
+__global__ void __launch_bounds__(128) append_kernel(KvView kv, uint16_t* k, uint16_t* v, int32_t* seq_lens,
+                                                     const uint16_t* k_new, const uint16_t* v_new) {
+  const int b = blockIdx.x;
+  const int L = seq_lens[b];
+  if (L < 0 || L >= kv.max_len) {
+    if (threadIdx.x == 0) report_error(kErrSeqLen);
+    return;  // uniform over the CTA
+  }
+  constexpr int U = D / 8;
+  for (int i = threadIdx.x; i < kv.hkv * U; i += blockDim.x) {
+    const int h = i / U, u = i - h * U;
+    const uint32_t row = kv.row(b, h, L);
+    if (row == kInvalidRow) continue;  // reported by row()
+    const int64_t src = ((int64_t)b * kv.hkv + h) * D + 8 * u;
+    *reinterpret_cast<uint4*>(k + (int64_t)row * D + 8 * u) = *reinterpret_cast<const uint4*>(k_new + src);
+    *reinterpret_cast<uint4*>(v + (int64_t)row * D + 8 * u) = *reinterpret_cast<const uint4*>(v_new + src);
+  }
+  __syncthreads();  // every thread has read seq_lens[b]
+  if (threadIdx.x == 0) seq_lens[b] = L + 1;
 }
 
 }  // namespace hga

@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (hga_attend, hga_build_summaries, hga_decode, hga_max_routed_tokens, hga_route,
+from . import (hga_append, hga_attend, hga_build_summaries, hga_decode, hga_max_routed_tokens, hga_route,
                hga_summary_bytes, make_kv, make_params)
 
 
@@ -78,6 +78,11 @@ class RoutedCache:
     # -- calls -------------------------------------------------------------------
     def build_summaries(self, stream=None) -> None:
         hga_build_summaries(self.kv, self.params, self.chunk_sum, self.group_sum, stream)
+
+    def append(self, k_new, v_new, stream=None) -> None:
+        """One more token per sequence (k_new, v_new: [B][Hkv][d] bfloat16 on the device); the lengths grow on
+        the device and a completed chunk's summaries are written (no host synchronisation: graph-capturable)."""
+        hga_append(self.kv, self.seq_lens, k_new, v_new, self.params, self.chunk_sum, self.group_sum, stream)
 
     def route(self, q, idx=None, n_idx=None, stream=None):
         q = self.q_tensor(q)

@@ -122,6 +122,26 @@ hga_status hga_build_summaries(const hga_kv* kv, const hga_params* p, void* chun
                                void* group_sum, cudaStream_t stream);
 
 /*
+ * Append one token to every sequence and keep the summaries current, for a
+ * decode loop that grows the cache (the incremental form of the summaries
+ * above; the pages keep summaries of the cached context up to date as it
+ * grows). For every sequence b:
+ *   K/V row k_new[b][h], v_new[b][h] -> position L = seq_lens[b] (contiguous
+ *   row, or slot L / page_size of the page table, whose page the caller has
+ *   assigned); then seq_lens[b] = L + 1, on the device; then, if L + 1 is a
+ *   multiple of chunk, the summaries of the chunk just completed, with the
+ *   same arithmetic as hga_build_summaries (bit-identical results).
+ *   k_new, v_new  [batch][n_kv_heads][head_dim] bfloat16, device
+ *   seq_lens      must be kv->seq_lens (updated in place)
+ * Two kernels on `stream`, no host synchronisation and no allocation, so the
+ * call can be captured in a CUDA graph together with hga_decode (call it once
+ * before capturing so its launch attributes are set). A sequence already at
+ * max_len is reported (device error bit 1) and left unchanged.
+ */
+hga_status hga_append(const hga_kv* kv, int32_t* seq_lens, const void* k_new, const void* v_new,
+                      const hga_params* p, void* chunk_sum, void* group_sum, cudaStream_t stream);
+
+/*
  * Upper bound on the routed tokens of one (sequence, KV head) over every
  * sequence length up to kv->max_len: the minimum idx_stride for hga_route,
  * hga_attend and hga_decode. Returns -1 on invalid arguments.
@@ -250,6 +270,31 @@ hga_status hga_prefill(const void* q, int32_t n_q_heads, int32_t n_queries, int3
 hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
                                const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
                                const hga_params* p, float* out, cudaStream_t stream);
+
+/*
+ * Growing-history chunked prefill: the same calls as hga_route_blocks /
+ * hga_prefill / hga_prefill_workspace_size, except that block b (queries at
+ * P_b = cache_len + b * block .. P_b + block - 1) routes over everything before
+ * it, [0, P_b), including the earlier blocks of the same call: its candidates
+ * are the full chunks of [0, P_b), its local chunk the last of them plus the
+ * partial tail up to P_b. Every query then attends its block's routed set plus
+ * the block's own tokens up to itself (causal), so the result is the decode
+ * rule applied block by block, as a drop-in for dense causal attention needs.
+ * Summaries must cover the full chunks of [0, cache_len + n_queries - block)
+ * (hga_build_summaries with seq_lens[0] = cache_len + n_queries, or hga_append
+ * as the tokens arrive). idx_stride / the workspace are sized for the longest
+ * list over the blocks (hga_prefill_growing_workspace_size).
+ */
+hga_status hga_route_blocks_growing(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                    const hga_kv* kv, int32_t cache_len, const void* chunk_sum,
+                                    const void* group_sum, const hga_params* p, int32_t* idx, int32_t idx_stride,
+                                    int32_t* n_idx, cudaStream_t stream);
+size_t hga_prefill_growing_workspace_size(const hga_kv* kv, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                                          int32_t cache_len, const hga_params* p);
+hga_status hga_prefill_growing(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,
+                               const hga_kv* kv, int32_t cache_len, const void* chunk_sum, const void* group_sum,
+                               const hga_params* p, float* out, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
 
 /*
  * Launch tuning, process-wide (not thread-safe against concurrent calls).
