@@ -164,6 +164,18 @@ def run_prefill(dev, steps: int, warmup: int):
     fl = prefill_flops(int(n_idx.sum().item()), nb * w.n_kv_heads)
     burst, sustained, kind = bf16_peak()
     attn_tf = fl / (attend * 1e-3) / 1e12
+
+    # growing history: block b routes over [0, 63488 + 64 b), earlier new blocks included
+    gwsb = hga.hga_prefill_growing_workspace_size(kv, w.n_q_heads, T, w.block, L0, p)
+    gws = torch.zeros(gwsb // 4, dtype=torch.int32, device=dev)
+    gstride = gwsb // (4 * nb * w.n_kv_heads) - 1
+    grow = timed(lambda: hga.hga_prefill_growing(q, w.n_q_heads, T, w.block, kv, L0, cs, gs, p, out, gws, gwsb),
+                 steps)
+    st, bits = hga.hga_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in growing prefill: {bits}")
+    g_routed = int(gws[nb * w.n_kv_heads * gstride: nb * w.n_kv_heads * (gstride + 1)].sum().item())
+    gfl = prefill_flops(g_routed, nb * w.n_kv_heads)
     return {
         "workload": "prefill_2048_on_63488: 2048 new tokens in 32 blocks of 64 on a 63488-token cache, 32 q / "
                     "4 KV heads, d 128, block-shared routing (C 128, g 16, top-32 + sink + local, top-4 groups) "
@@ -177,6 +189,10 @@ def run_prefill(dev, steps: int, warmup: int):
                      "unit": "TFLOP/s", "frac": round(attn_tf / burst, 4),
                      "frac_of_sustained": round(attn_tf / sustained, 4),
                      "traffic": profiled_traffic("prefill_64k_attn_kernel.md", PREFILL_SOURCES)},
+        "growing_history": {"what": "hga_prefill_growing: block b routes over its whole history "
+                                    "[0, 63488 + 64 b), earlier blocks of the call included",
+                            "ms_per_step": round(grow, 4), "tokens_per_s": round(T / (grow * 1e-3), 1),
+                            "flops_per_step": gfl, "tflops_step": round(gfl / (grow * 1e-3) / 1e12, 1)},
     }
 
 
@@ -409,6 +425,34 @@ def run_gpu(args, rank: int, world: int, dist):
     if st != 0:
         raise RuntimeError(f"device error in sweep: {bits}")
 
+    # serving loop: append one token per sequence + fused decode, replayed from a CUDA
+    # graph; the sequences start n_loop + warmup tokens short of 65536 and grow back to
+    # it (the appended token is the query's own; its K/V overwrite the cache's last rows)
+    n_loop = max(10, args.steps // 2)
+    cache.seq_lens.fill_(w.ctx_len - n_loop - args.warmup)
+    kn = torch.randn((B, w.n_kv_heads, w.head_dim), device=dev).to(torch.bfloat16)
+    vn = torch.randn((B, w.n_kv_heads, w.head_dim), device=dev).to(torch.bfloat16)
+    graph = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        cache.append(kn, vn)
+        cache.decode(q, out, lse)
+    for _ in range(args.warmup):
+        graph.replay()
+    loop_ms = timed(n_loop, graph.replay)
+    st, bits = hga.hga_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the decode loop: {bits}")
+    del graph
+    cache.seq_lens.copy_(lens_saved)
+    cache.build_summaries()
+    loop_step = statistics.median(loop_ms)
+    decode_loop = {"what": "hga_append + hga_decode captured in one CUDA graph, replayed per step "
+                           f"({n_loop} timed steps after {args.warmup}, lengths growing to {w.ctx_len}, "
+                           "L2 flushed between steps)",
+                   "us_per_step": round(loop_step * 1e3, 2), "queries_per_s": round(B / (loop_step * 1e-3)),
+                   "gpu_launches_per_step": 3}
+
     alg = B * decode_bytes(w.ctx_len)
     mean_launch_s = statistics.mean(times) / 1e3
     achieved = alg / mean_launch_s / 1e9
@@ -440,6 +484,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "latency_ms": {"p50": round(pct(50), 5), "p95": round(pct(95), 5), "p99": round(pct(99), 5)},
         "batch1_latency_us": round(statistics.median(lat) * 1e3, 2),
         "sweep": sweep,
+        "decode_loop_graph": decode_loop,
         "prefill": prefill,
     }
     return res, inp, w
