@@ -25,7 +25,7 @@ __all__ = [
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
     "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
-    "hga_prefill_growing_workspace_size", "hga_prefill_growing", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
+    "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
     "HGA_OPT_PREFILL_KERNEL", "STATUS_NAMES",
     "EXPORTED",
 ]
@@ -43,7 +43,7 @@ EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens",
             "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
             "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
             "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
-            "hga_prefill_growing_workspace_size", "hga_prefill_growing")
+            "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer")
 
 
 class HgaError(RuntimeError):
@@ -93,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "hga_route_blocks_growing": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, i32, vp, vp], i32),
         "hga_prefill_growing_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
         "hga_prefill_growing": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
+        "hga_host_kv_pointer": ([vp, ctypes.POINTER(vp)], i32),
         "hga_prefill_noalloc": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -253,6 +254,14 @@ def hga_prefill_growing(q, n_q_heads: int, n_queries: int, block: int, kv: hga_k
     _check(_lib.hga_prefill_growing(_addr(q), n_q_heads, n_queries, block, ctypes.byref(kv), cache_len,
                                     _addr(chunk_sum), _addr(group_sum), ctypes.byref(p), _addr(out),
                                     _addr(workspace), workspace_bytes, _stream(stream)), "hga_prefill_growing")
+
+
+def hga_host_kv_pointer(host_tensor) -> int:
+    """Device address of a pinned, mapped host buffer (a pinned CPU torch tensor or a raw address), for
+    hga_kv.k / hga_kv.v of a host-resident cache."""
+    dev = ctypes.c_void_p(0)
+    _check(_lib.hga_host_kv_pointer(_addr(host_tensor), ctypes.byref(dev)), "hga_host_kv_pointer")
+    return int(dev.value)
 
 
 def hga_set_launch_option(option: int, value: int) -> None:

@@ -731,6 +731,25 @@ hga_status hga_set_launch_option(int32_t option, int32_t value) {
   return HGA_ERR_INVALID_ARG;
 }
 
+hga_status hga_host_kv_pointer(const void* host, void** device_ptr) {
+  if (device_ptr == nullptr) return HGA_ERR_INVALID_ARG;
+  *device_ptr = nullptr;
+  if (host == nullptr) return HGA_ERR_INVALID_ARG;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, host) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return HGA_ERR_INVALID_ARG;
+  }
+  if (attr.type != cudaMemoryTypeHost) return HGA_ERR_INVALID_ARG;
+  void* dev = nullptr;
+  if (cudaHostGetDevicePointer(&dev, const_cast<void*>(host), 0) != cudaSuccess || dev == nullptr) {
+    cudaGetLastError();
+    return HGA_ERR_INVALID_ARG;
+  }
+  *device_ptr = dev;
+  return HGA_OK;
+}
+
 hga_status hga_get_device_error(cudaStream_t stream, int32_t* bits) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return HGA_ERR_CUDA;
   int v = 0;

@@ -318,6 +318,20 @@ enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2, HGA_OPT_PREFILL_KER
 hga_status hga_set_launch_option(int32_t option, int32_t value);
 
 /*
+ * Host-resident K/V (the pages' own placement: the full cache in host memory,
+ * only the routed working set moved to the GPU). K and V may live in pinned,
+ * mapped host memory (cudaHostAlloc, or cudaHostRegister with the mapped
+ * flag); this call returns the device address of such a buffer, to be put in
+ * hga_kv.k / hga_kv.v. The routing summaries stay in device memory. Every call
+ * then reads K/V through the host link (PCIe or NVLink-C2C): hga_decode and
+ * hga_route / hga_attend read only the routed rows, hga_build_summaries and
+ * hga_append read and write what they always do. Returns HGA_ERR_INVALID_ARG
+ * (and *device_ptr = NULL) when `host` is not pinned and mapped for the
+ * current device, so an unmapped address never reaches a kernel.
+ */
+hga_status hga_host_kv_pointer(const void* host, void** device_ptr);
+
+/*
  * Synchronise `stream`, then read and clear this device's error word.
  * HGA_OK if no kernel reported a problem since the last call,
  * HGA_ERR_DEVICE_FAULT for a bad device-side input, HGA_ERR_TIMEOUT for an
