@@ -9,7 +9,8 @@ The arithmetic is in ``hga_oracle.c`` (plain C, double precision); this module
 compiles it with gcc and wraps each function for numpy arrays. Each wrapper names
 the step of the method it states: chunk/group summaries, head-summed routing
 scores, chunk top-k with sink and local chunks kept, group top-G, exact softmax
-attention over the routed set, and the block-shared routing of chunked prefill.
+attention over the routed set, the block-shared routing of chunked prefill, and
+the block-then-token variant (top blocks, then top tokens inside them).
 """
 from __future__ import annotations
 
@@ -60,6 +61,8 @@ def lib():
         L.oracle_attend.restype = None
         L.oracle_prefill_block.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp, i32, i32, dbl, vp]
         L.oracle_prefill_block.restype = None
+        L.oracle_hisa_route.argtypes = [vp, i32, i32, vp, vp, i32, i32, i32, i32, vp, i32, vp]
+        L.oracle_hisa_route.restype = i32
         _lib = L
     return _lib
 
@@ -150,6 +153,38 @@ def route(q, chunk_sum, group_sum, L: int, C: int, g: int, k: int, G: int, retur
     if n < 0:
         raise RuntimeError("oracle_route_block: capacity")
     return (tok[:n].copy(), kept[:nk.value].copy()) if return_chunks else tok[:n].copy()
+
+
+def hisa_candidates(L: int, C: int, m: int) -> int:
+    """Tokens the block-then-token route scores for one query: first block + top-m blocks + last block
+    and tail (every token when nf <= 2)."""
+    nf = L // C
+    if nf <= 2:
+        return L
+    return C + min(m, nf - 2) * C + (L - (nf - 1) * C)
+
+
+def hisa_route(q, chunk_sum, K, L: int, C: int, m: int, k_tok: int, return_scored: bool = False):
+    """Block-then-token routed positions (ascending) of one decode query q [R][d] over K [L][d]: the
+    top-m chunks (plus the first and last) by their summaries, then the top k_tok tokens inside them."""
+    q = _u16(q)
+    R, d = q.shape
+    K = _u16(K)
+    if K.shape[0] < L:
+        raise IndexError("K shorter than L")
+    cap = max(min(k_tok, hisa_candidates(L, C, m)), 1)
+    tok = np.zeros(cap, dtype=np.int32)
+    scored = ctypes.c_int64(0)
+    n = lib().oracle_hisa_route(_p(q), R, d, _p(_u16(chunk_sum)), _p(K), L, C, m, k_tok, _p(tok), cap,
+                                ctypes.byref(scored))
+    if n < 0:
+        raise RuntimeError("oracle_hisa_route: capacity")
+    return (tok[:n].copy(), int(scored.value)) if return_scored else tok[:n].copy()
+
+
+def token_scores(q, K) -> np.ndarray:
+    """Head-summed indexer score of every key row of K [n][d] for q [R][d] (the token step's score)."""
+    return chunk_scores(q, K)
 
 
 def attend(q, K, V, tokens, scale: float | None = None, with_lse: bool = False):

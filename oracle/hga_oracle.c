@@ -25,7 +25,11 @@
  *   - the routing score of a KV head is the sum over the query heads that share
  *     it, without the softmax scale; ties go to the lower index;
  *   - prefill blocks share one routing decision: the score is the maximum over
- *     the block's queries of the head-summed score.
+ *     the block's queries of the head-summed score;
+ *   - the block-then-token variant (oracle_hisa_route) uses the chunks as its
+ *     blocks and the same head-summed score for blocks and tokens; the first
+ *     and last blocks are always among the kept blocks, and the token step
+ *     chooses among all kept blocks' tokens.
  *
  * Parity pins for every function are in tests/test_oracle_pins.py.
  */
@@ -263,6 +267,76 @@ int32_t oracle_route(const uint16_t* q, int32_t R, int32_t d, const uint16_t* ch
                      int32_t* tokens, int32_t cap) {
   return oracle_route_block(q, 1, (int64_t)R * d, R, d, chunk_sum, group_sum, L, C, g, k, G, tokens,
                             cap, NULL, NULL);
+}
+
+/* ------------------------------------------------- block-then-token routing */
+
+/*
+ * Block-then-token routing of one decode query (the HISA article's two steps,
+ * "Hierarchical Indexing Sparse Attention", shijienb.com summary: a coarse
+ * filter on per-block feature vectors keeps the best blocks, always with the
+ * start and the end of the text, then token-level scoring runs only inside the
+ * kept blocks). Blocks are the chunks of size C with the same summaries, and the
+ * scoring rule is the head-summed one of oracle_route:
+ *   nf <= 2 -> candidates: every token [0, L)
+ *   else    -> candidates: [0, C) (first block) + the tokens of the top
+ *              min(m, nf-2) chunks among 1..nf-2 (score desc, id asc) +
+ *              [(nf-1)*C, L) (last block and partial tail)
+ *   token score tau_t = sum over the R heads of q_i . K_t (double); keep the
+ *   top min(k_tok, n_cand) candidates by (tau desc, t asc), written ascending.
+ *   K [L][d] holds the keys of this (sequence, KV head).
+ * Returns the kept count, -1 if cap is too small. *n_scored (optional) gets the
+ * number of scored vectors (the cost the article's O(L^2/B + L m B) counts over
+ * a whole prefill): (nf - 2) summaries + n_cand tokens when nf > 2, n_cand
+ * otherwise.
+ */
+int32_t oracle_hisa_route(const uint16_t* q, int32_t R, int32_t d, const uint16_t* chunk_sum, const uint16_t* K,
+                          int32_t L, int32_t C, int32_t m, int32_t k_tok, int32_t* tokens, int32_t cap,
+                          int64_t* n_scored) {
+  int32_t nf = L / C;
+  int32_t* cand_tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+  int32_t n_cand = 0;
+  int64_t scored_vectors = 0;
+  if (nf <= 2) {
+    for (int32_t t = 0; t < L; ++t) cand_tok[n_cand++] = t;
+  } else {
+    int32_t n_blk = nf - 2;
+    int32_t r = m < n_blk ? m : n_blk;
+    scored* blk = (scored*)malloc(sizeof(scored) * (size_t)n_blk);
+    int32_t* chosen = (int32_t*)malloc(sizeof(int32_t) * (size_t)(r > 0 ? r : 1));
+    for (int32_t c = 1; c <= nf - 2; ++c) {
+      blk[c - 1].score = route_score(q, 1, (int64_t)R * d, R, d, chunk_sum + (int64_t)c * d);
+      blk[c - 1].id = c;
+    }
+    scored_vectors += n_blk;
+    qsort(blk, (size_t)n_blk, sizeof(scored), by_score_desc);
+    for (int32_t i = 0; i < r; ++i) chosen[i] = blk[i].id;
+    qsort(chosen, (size_t)r, sizeof(int32_t), by_int_asc);
+    for (int32_t t = 0; t < C; ++t) cand_tok[n_cand++] = t; /* first block */
+    for (int32_t i = 0; i < r; ++i)
+      for (int32_t t = 0; t < C; ++t) cand_tok[n_cand++] = chosen[i] * C + t;
+    for (int32_t t = (nf - 1) * C; t < L; ++t) cand_tok[n_cand++] = t; /* last block + tail */
+    free(blk);
+    free(chosen);
+  }
+  scored_vectors += n_cand;
+  if (n_scored) *n_scored = scored_vectors;
+  int32_t keep = k_tok < n_cand ? k_tok : n_cand;
+  if (keep > cap) {
+    free(cand_tok);
+    return -1;
+  }
+  scored* tok = (scored*)malloc(sizeof(scored) * (size_t)(n_cand > 0 ? n_cand : 1));
+  for (int32_t i = 0; i < n_cand; ++i) {
+    tok[i].score = route_score(q, 1, (int64_t)R * d, R, d, K + (int64_t)cand_tok[i] * d);
+    tok[i].id = cand_tok[i];
+  }
+  qsort(tok, (size_t)n_cand, sizeof(scored), by_score_desc);
+  for (int32_t i = 0; i < keep; ++i) tokens[i] = tok[i].id;
+  qsort(tokens, (size_t)keep, sizeof(int32_t), by_int_asc);
+  free(tok);
+  free(cand_tok);
+  return keep;
 }
 
 /* -------------------------------------------------------------- attention */

@@ -358,3 +358,96 @@ def test_prefill_full_coverage_is_dense_causal():
     for p in range(nq):
         want = dense_attention(qf[p], Kf[: L0 + p + 1], Vf[: L0 + p + 1], 1 / math.sqrt(d))
         np.testing.assert_allclose(out[p], want, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------- block-then-token routing
+
+
+def brute_hisa(q_f64, cs_f64, K_f64, L, C, m, k_tok):
+    """Block-then-token routing by direct enumeration and Python sorting."""
+    nf = L // C
+    hs = q_f64.sum(axis=0)
+
+    def score(v):
+        return float(sum(hs[e] * v[e] for e in range(len(v))))
+
+    if nf <= 2:
+        cand = list(range(L))
+    else:
+        blocks = sorted(range(1, nf - 1), key=lambda c: (-score(cs_f64[c]), c))
+        kept = sorted(blocks[:m])
+        cand = list(range(C)) + [c * C + t for c in kept for t in range(C)] + list(range((nf - 1) * C, L))
+    order = sorted(cand, key=lambda t: (-score(K_f64[t]), t))
+    return sorted(order[:k_tok])
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_hisa_route_matches_brute_force(seed):
+    rng = np.random.default_rng(300 + seed)
+    C = int(rng.choice([8, 16, 32]))
+    L = int(rng.integers(1, 12 * C))
+    d = int(rng.choice([8, 16]))
+    R = int(rng.integers(1, 5))
+    m = int(rng.integers(1, 6))
+    k_tok = int(rng.integers(1, 4 * C))
+    K = rand_bf16(rng, (L, d))
+    q = rand_bf16(rng, (R, d))
+    cs, _ = oracle.summaries(K, C, 4)
+    got, scored = oracle.hisa_route(q, cs, K, L, C, m, k_tok, return_scored=True)
+    want = brute_hisa(oracle.bf16_to_f64(q), oracle.bf16_to_f64(cs), oracle.bf16_to_f64(K), L, C, m, k_tok)
+    assert got.tolist() == want
+    nf = L // C
+    n_cand = oracle.hisa_candidates(L, C, m)
+    assert len(got) == min(k_tok, n_cand)
+    # the work the article's cost model counts: block summaries scored + candidate tokens scored
+    assert scored == (nf - 2 if nf > 2 else 0) + n_cand
+
+
+def test_hisa_full_coverage_keeps_every_token():
+    rng = np.random.default_rng(7)
+    L, C, d = 10 * 16 + 5, 16, 8
+    K = rand_bf16(rng, (L, d))
+    q = rand_bf16(rng, (3, d))
+    cs, _ = oracle.summaries(K, C, 4)
+    assert oracle.hisa_route(q, cs, K, L, C, 100, 10 * L).tolist() == list(range(L))
+
+
+def test_hisa_ties_go_to_lower_position():
+    # identical keys: every block and token score ties, so the lowest blocks and
+    # then the lowest positions are kept
+    L, C, d, m, k_tok = 8 * 16, 16, 8, 2, 20
+    K = to_bf16_bits(np.ones((L, d)))
+    q = to_bf16_bits(np.ones((2, d)))
+    cs, _ = oracle.summaries(K, C, 4)
+    assert oracle.hisa_route(q, cs, K, L, C, m, k_tok).tolist() == list(range(20))
+
+
+def test_hisa_keeps_the_highest_scoring_candidates():
+    # one key per candidate block made clearly highest along q: the token step must
+    # keep exactly those (and the rest of the kept set scores no higher than them)
+    rng = np.random.default_rng(11)
+    L, C, d = 12 * 16, 16, 16
+    Kf = rng.standard_normal((L, d)) * 0.1
+    qf = np.zeros((1, d))
+    qf[0, 0] = 1.0
+    hot = [3, 70, 150, 190]  # first block, two middle blocks, the last block
+    for t in hot:
+        Kf[t, 0] = 4.0
+    K = (torch.from_numpy(Kf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    q = to_bf16_bits(qf)
+    cs, _ = oracle.summaries(K, C, 4)
+    got = oracle.hisa_route(q, cs, K, L, C, 3, len(hot)).tolist()
+    assert got == hot
+
+
+def test_hisa_cost_matches_the_articles_model():
+    # Summed over the queries of a long prefill, the scored vectors per query,
+    # (L/C - 2) summaries + (m + 2) C tokens (+ the tail), total about
+    # N^2 / (2C) + N (m + 2) C: the article's O(L^2/B + L m B) with B = C.
+    C, m, N = 128, 32, 65536
+    total = 0
+    for L in range(1, N + 1):
+        nf = L // C
+        total += (nf - 2 if nf > 2 else 0) + oracle.hisa_candidates(L, C, m)
+    model = N * N / (2 * C) + N * (m + 2) * C
+    assert abs(total / model - 1.0) < 0.02
