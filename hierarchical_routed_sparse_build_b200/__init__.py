@@ -25,7 +25,8 @@ __all__ = [
     "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
     "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
-    "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer", "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
+    "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer", "hga_decode_hisa", "hga_max_hisa_tokens",
+    "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
     "HGA_OPT_PREFILL_KERNEL", "STATUS_NAMES",
     "EXPORTED",
 ]
@@ -43,7 +44,8 @@ EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens",
             "hga_attend", "hga_decode", "hga_set_launch_option", "hga_get_device_error",
             "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
             "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
-            "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer")
+            "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer",
+            "hga_decode_hisa", "hga_max_hisa_tokens")
 
 
 class HgaError(RuntimeError):
@@ -94,6 +96,8 @@ def _load() -> ctypes.CDLL:
         "hga_prefill_growing_workspace_size": ([KV, i32, i32, i32, i32, P], sz),
         "hga_prefill_growing": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp, sz, vp], i32),
         "hga_host_kv_pointer": ([vp, ctypes.POINTER(vp)], i32),
+        "hga_decode_hisa": ([vp, i32, KV, vp, P, i32, vp, vp, vp, i32, vp, vp], i32),
+        "hga_max_hisa_tokens": ([KV, P, i32], i32),
         "hga_prefill_noalloc": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -262,6 +266,21 @@ def hga_host_kv_pointer(host_tensor) -> int:
     dev = ctypes.c_void_p(0)
     _check(_lib.hga_host_kv_pointer(_addr(host_tensor), ctypes.byref(dev)), "hga_host_kv_pointer")
     return int(dev.value)
+
+
+def hga_decode_hisa(q, n_q_heads: int, kv: hga_kv, chunk_sum, p: hga_params, top_tokens: int, out, lse=None,
+                    idx=None, idx_stride: int = 0, n_idx=None, stream=None) -> None:
+    """Block-then-token routed decode: top chunks by summary, then the top_tokens tokens inside them."""
+    _check(_lib.hga_decode_hisa(_addr(q), n_q_heads, ctypes.byref(kv), _addr(chunk_sum), ctypes.byref(p),
+                                top_tokens, _addr(out), _addr(lse), _addr(idx), idx_stride, _addr(n_idx),
+                                _stream(stream)), "hga_decode_hisa")
+
+
+def hga_max_hisa_tokens(kv: hga_kv, p: hga_params, top_tokens: int) -> int:
+    n = _lib.hga_max_hisa_tokens(ctypes.byref(kv), ctypes.byref(p), top_tokens)
+    if n < 0:
+        raise HgaError(1, "hga_max_hisa_tokens")
+    return n
 
 
 def hga_set_launch_option(option: int, value: int) -> None:

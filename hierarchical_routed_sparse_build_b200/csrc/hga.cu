@@ -15,6 +15,7 @@
 #include "hga.h"
 #include "hga_common.cuh"
 #include "hga_decode.cuh"
+#include "hga_hisa.cuh"
 #include "hga_prefill_attn.cuh"
 #include "hga_prefill_attn2.cuh"
 #include "hga_prefill_route.cuh"
@@ -396,6 +397,55 @@ hga_status noalloc_area(void** out) {
   return HGA_OK;
 }
 
+template <int D>
+cudaError_t launch_hisa(const RoutedArgs& a, int units, int P, int smem_bytes, cudaStream_t stream) {
+  auto kern = hisa_decode_kernel<D>;
+  static std::atomic<int> smem_set[kMaxDevices];
+  static std::atomic<bool> np_set[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (smem_bytes > smem_set[dev].load()) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess) return e;
+    smem_set[dev].store(smem_bytes);
+  }
+  if (P > 8 && !np_set[dev].load()) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    np_set[dev].store(true);
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3((unsigned)(units * P), 1, 1);
+  cfg.blockDim = dim3(kRoutedThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Kept tokens of the block-then-token route at the longest context (the list
+// length hga_decode_hisa writes is at most this).
+int hisa_max_routed(const hga_kv* kv, const hga_params* p, int32_t top_tokens) {
+  const int C = p->chunk, nf = kv->max_len / C;
+  int most = 0;  // most candidates over lengths <= max_len
+  for (int L = kv->max_len; L >= 0 && L > kv->max_len - 2 * C; --L) {
+    const int f = L / C;
+    const int n = f <= 2 ? L : C + (f - 2 < p->top_chunks ? f - 2 : p->top_chunks) * C + (L - (f - 1) * C);
+    if (n > most) most = n;
+  }
+  (void)nf;
+  return most < top_tokens ? most : top_tokens;
+}
+
 }  // namespace
 }  // namespace hga
 
@@ -568,6 +618,47 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
   if (g_decode_kernel.load() != 1 && p->group % 16 == 0)
     return run_decode(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
   return run_routed<kModeDecode>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+int32_t hga_max_hisa_tokens(const hga_kv* kv, const hga_params* p, int32_t top_tokens) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK || top_tokens < 1) return -1;
+  return hisa_max_routed(kv, p, top_tokens);
+}
+
+hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                           const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,
+                           int32_t idx_stride, int32_t* n_idx, cudaStream_t stream) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || !aligned16(chunk_sum) || out == nullptr ||
+      top_tokens < 1)
+    return HGA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
+  if (idx != nullptr && idx_stride < hisa_max_routed(kv, p, top_tokens)) return HGA_ERR_INVALID_ARG;
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.kv = make_kv_view(kv);
+  a.sv = make_sum_view(kv, p, chunk_sum, nullptr);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  routing_args(a, kv, p);
+  a.k_tok = top_tokens;
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.out = out;
+  a.lse = lse;
+  a.idx_out = idx;
+  a.n_idx_out = n_idx;
+  a.idx_stride = idx ? idx_stride : 0;
+  const int smem = HisaSmem(kv->head_dim, a.n_pad, a.kcap, hisa_tok_pad(p->chunk, a.kcap), top_tokens).total;
+  if (smem > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
+  const int units = kv->batch * kv->n_kv_heads;
+  const int P = pick_cluster(units);
+  cudaError_t e = kv->head_dim == 128 ? launch_hisa<128>(a, units, P, smem, stream)
+                                      : launch_hisa<64>(a, units, P, smem, stream);
+  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
 }
 
 hga_status hga_route_blocks(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,

@@ -60,6 +60,7 @@ struct RoutedArgs {
   int C, g, k, G;     // routing parameters (G already <= C/g)
   int n_pad;          // >= max candidates (max_chunks - 2), >= 2
   int kcap;           // >= kept chunks for any length (min(k, max_chunks - 2)), >= 1
+  int k_tok;          // block-then-token routing: tokens kept by the token step
   float scale_log2;   // softmax scale * log2(e)
   float* out;         // [B][Hq][D]
   float* lse;         // [B][Hq] or null

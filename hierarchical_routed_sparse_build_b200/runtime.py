@@ -9,8 +9,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (hga_append, hga_attend, hga_build_summaries, hga_decode, hga_max_routed_tokens, hga_route,
-               hga_summary_bytes, make_kv, make_params)
+from . import (hga_append, hga_attend, hga_build_summaries, hga_decode, hga_decode_hisa, hga_max_hisa_tokens,
+               hga_max_routed_tokens, hga_route, hga_summary_bytes, make_kv, make_params)
 
 
 def _dev_u16(a: np.ndarray, device) -> torch.Tensor:
@@ -78,6 +78,22 @@ class RoutedCache:
     # -- calls -------------------------------------------------------------------
     def build_summaries(self, stream=None) -> None:
         hga_build_summaries(self.kv, self.params, self.chunk_sum, self.group_sum, stream)
+
+    def decode_hisa(self, q, top_tokens: int, out=None, lse=None, want_idx: bool = False, stream=None):
+        """Block-then-token routed decode (top chunks by summary, then the top_tokens tokens inside them)."""
+        q = self.q_tensor(q)
+        if out is None:
+            out, lse = self.out_buffers()
+        idx = n_idx = None
+        stride = 0
+        if want_idx:
+            stride = hga_max_hisa_tokens(self.kv, self.params, top_tokens)
+            idx = torch.full((self.batch, self.n_kv_heads, max(stride, 1)), -1, dtype=torch.int32,
+                             device=self.device)
+            n_idx = torch.zeros((self.batch, self.n_kv_heads), dtype=torch.int32, device=self.device)
+        hga_decode_hisa(q, self.n_q_heads, self.kv, self.chunk_sum, self.params, top_tokens, out, lse, idx,
+                        max(stride, 1) if want_idx else 0, n_idx, stream)
+        return (out, lse, idx, n_idx) if want_idx else (out, lse)
 
     def append(self, k_new, v_new, stream=None) -> None:
         """One more token per sequence (k_new, v_new: [B][Hkv][d] bfloat16 on the device); the lengths grow on

@@ -272,6 +272,31 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
                                const hga_params* p, float* out, cudaStream_t stream);
 
 /*
+ * Block-then-token routed decode (the HISA article's two steps: a coarse filter
+ * on per-block feature vectors keeps the best blocks, always with the beginning
+ * and the end of the text, then token-level scoring runs only inside the kept
+ * blocks, taking the indexer's O(L^2) cost to O(L^2/B + L m B)). Blocks are the
+ * chunks, with the summaries of hga_build_summaries (only chunk_sum is read),
+ * and both steps use the head-summed score of hga_route. Per sequence b and KV
+ * head h with nf = seq_lens[b] / chunk full chunks:
+ *   candidates = every token [0, L) when nf <= 2; else [0, C) + the tokens of
+ *   the top p->top_chunks chunks among 1..nf-2 (score desc, lower id first)
+ *   + [(nf-1)*C, L)
+ *   kept = the top_tokens candidates by tau_t = sum_i q_i . K_t (desc, lower
+ *   position first), all of them if there are no more than top_tokens
+ *   out/lse = exact softmax attention over the kept tokens, as hga_attend.
+ * idx/n_idx (optional, as hga_decode) receive the kept positions, ascending;
+ * idx_stride >= hga_max_hisa_tokens(kv, p, top_tokens). p->group and
+ * p->top_groups must be valid as for hga_route but are not used.
+ */
+hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                           const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,
+                           int32_t idx_stride, int32_t* n_idx, cudaStream_t stream);
+
+/* Most positions hga_decode_hisa keeps for one (sequence, KV head); -1 on invalid arguments. */
+int32_t hga_max_hisa_tokens(const hga_kv* kv, const hga_params* p, int32_t top_tokens);
+
+/*
  * Growing-history chunked prefill: the same calls as hga_route_blocks /
  * hga_prefill / hga_prefill_workspace_size, except that block b (queries at
  * P_b = cache_len + b * block .. P_b + block - 1) routes over everything before

@@ -112,3 +112,40 @@ def assert_lse_close(gpu: np.ndarray, ref: np.ndarray, what: str) -> None:
 
 def scale_for(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def check_hisa_route(tokens: np.ndarray, q_heads: np.ndarray, cs: np.ndarray, K: np.ndarray, L: int, C: int,
+                     m: int, k_tok: int, what: str = "hisa route") -> bool:
+    """Check a block-then-token list against oracle.hisa_route on the same summaries and keys.
+
+    Returns True when it equals the oracle's list. Otherwise it must have the oracle's length, be
+    ascending inside [0, L), come from allowed blocks (first, last + tail, or a middle block scoring
+    within the near-tie rule of the block boundary) and, when its visible blocks are the oracle's,
+    be a top-k_tok of the oracle's candidates under the near-tie rule.
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    want = oracle.hisa_route(q_heads, cs, K, L, C, m, k_tok)
+    if tokens.shape == want.shape and np.array_equal(tokens, want):
+        return True
+    assert tokens.size == want.size, f"{what}: size {tokens.size} != {want.size}"
+    assert np.all(np.diff(tokens) > 0) and tokens.min() >= 0 and tokens.max() < L, f"{what}: not a valid list"
+    nf = L // C
+    tau = oracle.token_scores(q_heads, np.ascontiguousarray(K[:L]))
+    if nf <= 2:
+        cands = list(range(L))
+    else:
+        cscore = oracle.chunk_scores(q_heads, cs[:nf])
+        r = min(m, nf - 2)
+        order = sorted(range(1, nf - 1), key=lambda c: (-cscore[c], c))
+        kept = set(order[:r])
+        visible = {int(t) // C for t in tokens if C <= t < (nf - 1) * C}
+        if r < nf - 2:
+            s_r, s_r1 = cscore[order[r - 1]], cscore[order[r]]
+            tol = TIE_REL * max(abs(s_r), 1e-6)
+            for c in visible:
+                assert cscore[c] >= s_r1 - tol, f"{what}: block {c} is not among the top blocks"
+        if not visible <= kept:
+            return False  # a near-tie block swap: the token step ran on other candidates
+        cands = list(range(C)) + [c * C + t for c in sorted(kept) for t in range(C)] + list(range((nf - 1) * C, L))
+    _check_selection({t: tau[t] for t in cands}, set(tokens.tolist()), tokens.size, what + " tokens")
+    return False
