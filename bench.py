@@ -65,6 +65,26 @@ DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh", "hga_
 PREFILL_SOURCES = ("hga_common.cuh", "hga_tcgen05.cuh", "hga_prefill_attn.cuh")
 
 
+HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (the DSA indexer's top-k)
+
+
+def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64) -> int:
+    """Algorithmic HBM bytes of one block-then-token decode query (all KV heads): candidate chunk
+    summaries, K of every candidate token (the token step scores them), K and V of the kept tokens,
+    q, out and lse."""
+    C, d, hkv, hq = w.chunk, w.head_dim, w.n_kv_heads, w.n_q_heads
+    nf = L // C
+    if nf <= 2:
+        cand, n_ct = 0, L
+    else:
+        cand = nf - 2
+        n_ct = C + min(w.top_chunks, cand) * C + (L - (nf - 1) * C)
+    kept = min(k_tok, n_ct)
+    scored_k = n_ct if n_ct > k_tok else 0
+    return (cand * hkv * d * 2 + scored_k * hkv * d * 2 + kept * hkv * d * 2 * 2
+            + hq * d * 2 + hq * d * 4 + hq * 4)
+
+
 def kernel_source_hash(names=DECODE_SOURCES) -> str:
     """sha256 (first 16 hex) of the device-code files one kernel is built from."""
     import hashlib
@@ -448,6 +468,23 @@ def run_gpu(args, rank: int, world: int, dist):
     cache.build_summaries()
     loop_step = statistics.median(loop_ms)
 
+    # block-then-token decode (HISA indexer variant) on the same cache: top-32 chunks,
+    # then the top 2048 tokens of their 4352 candidates
+    hisa_ms = timed(max(10, args.steps // 2),
+                    lambda: cache.decode_hisa(q, HISA_TOKENS, out, lse))
+    st, bits = hga.hga_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the block-then-token decode: {bits}")
+    hisa_step = statistics.median(hisa_ms)
+    hbm_peak, _ = peaks()
+    hisa = {"what": "hga_decode_hisa: top-32 chunks by summary (plus first and last), then the top "
+                    f"{HISA_TOKENS} of their tokens by the head-summed indexer score, exact attention over them; "
+                    f"{B} x 64K sequences",
+            "us_per_step": round(hisa_step * 1e3, 2), "queries_per_s": round(B / (hisa_step * 1e-3)),
+            "alg_bytes_per_query": hisa_bytes(w.ctx_len),
+            "GB_s": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9, 1),
+            "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4)}
+
     # host-resident K/V (the pages' placement): 8 of the sequences in pinned, mapped host
     # memory, summaries in HBM; the decode kernel reads only the routed rows over the host link
     Bh = min(B, 8)
@@ -509,6 +546,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "sweep": sweep,
         "decode_loop_graph": decode_loop,
         "host_resident_kv": host_kv,
+        "block_then_token": hisa,
         "prefill": prefill,
     }
     return res, inp, w
