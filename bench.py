@@ -65,7 +65,7 @@ DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh", "hga_
 PREFILL_SOURCES = ("hga_common.cuh", "hga_tcgen05.cuh", "hga_prefill_attn.cuh")
 
 
-HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (the DSA indexer's top-k)
+HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (below the 2304 the two-level route keeps)
 
 
 def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64) -> int:

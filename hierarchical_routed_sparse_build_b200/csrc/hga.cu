@@ -637,6 +637,7 @@ hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, c
     return HGA_ERR_INVALID_ARG;
   if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
   if (idx != nullptr && idx_stride < hisa_max_routed(kv, p, top_tokens)) return HGA_ERR_INVALID_ARG;
+  if (p->chunk % 16 != 0) return HGA_ERR_UNSUPPORTED;  // token batches of 16 stay inside one chunk
   RoutedArgs a;
   std::memset(&a, 0, sizeof a);
   a.kv = make_kv_view(kv);

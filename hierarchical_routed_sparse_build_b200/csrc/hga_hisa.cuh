@@ -17,12 +17,14 @@
 //   --  cluster barrier
 //   R2  top-m chunks (bucket select, ascending ids), in every CTA
 //   T1  the candidate tokens, [0, C) + the kept chunks' tokens + [(nf-1)C, L)
-//       (every token when nf <= 2), are split over the CTAs and scored the
-//       same way in 16-row batches of K; their 64-bit keys (score bits, then
-//       lower position) go to every CTA
+//       (every token when nf <= 2), are split over the CTAs in batches of 16
+//       consecutive positions and scored the same way from registers; their
+//       64-bit keys (score bits, then lower position) and the score range go
+//       to every CTA
 //   --  cluster barrier (skipped, with T1 and T2, when the candidates are no
 //       more than the tokens to keep)
-//   T2  top k_tok tokens (bucket select, ascending positions), in every CTA
+//   T2  top k_tok tokens (select_top_tokens, ascending positions), in every
+//       CTA
 //   A   exact attention over the kept tokens: 16-token tiles split over the
 //       CTAs and round-robin over the warps (hga_attention.cuh), rows staged
 //       in batches of kEntryBatch entries
@@ -37,8 +39,8 @@ namespace hga {
 // union region holds the chunk keys, the token keys and the select scratch,
 // then the per-warp attention tiles, then the per-warp partial outputs.
 struct HisaSmem {
-  int qsum, sel, pages, red_m, red_l, cta_o, cta_m, cta_l, qfrag, hist, misc, rows, tsel, uni, ckeys, tkeys,
-      scratch, tiles, red_o, total;
+  int qsum, sel, pages, red_m, red_l, cta_o, cta_m, cta_l, qfrag, hist, misc, kred, tmm, rows, tsel, uni, ckeys,
+      tkeys, scratch, tiles, red_o, total;
   __host__ __device__ static int up16(int x) { return (x + 15) & ~15; }
   // n_tok_pad >= the most candidate tokens at any length, k_tok = tokens kept
   __host__ __device__ HisaSmem(int D, int n_pad, int kcap, int n_tok_pad, int k_tok) {
@@ -54,6 +56,8 @@ struct HisaSmem {
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
     hist = o;    o = up16(o + 4 * kBuckets);
     misc = o;    o = up16(o + 4 * 32);
+    kred = o;    o = up16(o + 8 * (2 * kRoutedWarps + 2));
+    tmm = o;     o = up16(o + 4 * 2 * (kGatherSlots + kRoutedWarps));
     rows = o;    o = up16(o + 4 * kEntryBatch);
     tsel = o;    o = up16(o + 4 * k_tok);
     uni = o;
@@ -71,6 +75,173 @@ struct HisaSmem {
     total = o;
   }
 };
+
+constexpr int kTokRankCap = 128;  // boundary keys ranked pairwise in the token select
+constexpr int kTokRefine = 8;     // key-range refinements before the pairwise ranking (7 suffice)
+
+// dot8 with one packed fp32 FMA per bf16 pair: even elements accumulate in .x,
+// odd ones in .y, each rounding exactly like the scalar fmaf chain of dot8.
+__device__ __forceinline__ float dot8_x2(const uint4 x, const float (&q)[8]) {
+  float2 s = __fmul2_rn(make_float2(bf16_lo(x.x), bf16_hi(x.x)), make_float2(q[0], q[1]));
+  s = __ffma2_rn(make_float2(bf16_lo(x.y), bf16_hi(x.y)), make_float2(q[2], q[3]), s);
+  s = __ffma2_rn(make_float2(bf16_lo(x.z), bf16_hi(x.z)), make_float2(q[4], q[5]), s);
+  s = __ffma2_rn(make_float2(bf16_lo(x.w), bf16_hi(x.w)), make_float2(q[6], q[7]), s);
+  return s.x + s.y;
+}
+
+// Score of a route key (inverse of float_order_bits on the upper word).
+__device__ __forceinline__ float route_key_score(uint64_t key) {
+  const uint32_t u = (uint32_t)(key >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+// Warp 0 walks the histogram from the top bucket down and finds the bucket
+// holding the need-th key: misc[0] = that bucket, misc[1] = keys above it.
+__device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, int* misc) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  constexpr int PER = kBuckets / 32;
+  int tot = 0;
+  for (int k = 0; k < PER; ++k) tot += hist[kBuckets - 1 - PER * lane - k];
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int excl = incl - tot;
+  if (excl < need && need <= incl) {
+    int acc = excl;
+    for (int k = 0; k < PER; ++k) {
+      const int bk = kBuckets - 1 - PER * lane - k;
+      if (acc + hist[bk] >= need) {
+        misc[0] = bk;
+        misc[1] = acc;
+        break;
+      }
+      acc += hist[bk];
+    }
+  }
+}
+
+// Top r of n distinct route keys (1 <= r < n), written to sel[] as their ids in
+// the keys' storage order (the token keys are stored in ascending position, so
+// the kept positions come out ascending). lo and hi are the least and greatest
+// score among the keys. The first histogram cuts [lo, hi] into kBuckets equal
+// score intervals, which for a bell-shaped score distribution leaves a few
+// dozen keys in the bucket holding the r-th key whatever r is (cutting the
+// order-preserving bit pattern instead crowds most keys into the few buckets
+// of the typical magnitude). While that boundary bucket holds more than
+// kTokRankCap keys, its key range is cut again into kBuckets equal intervals
+// of the 64-bit key; the boundary keys are then ranked pairwise. Every bucket
+// map is monotone in the key, so a bucket is a contiguous key range and the
+// kept set equals a full sort's. kred: 2 * kRoutedWarps + 2 words.
+__device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, int r, float lo, float hi, int* sel,
+                                                  int* hist, int* misc, uint64_t* scratch, uint64_t* kred) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float vscale = hi > lo ? (float)kBuckets / (hi - lo) : 0.f;
+  auto vbucket = [&](uint64_t key) {
+    return min(kBuckets - 1, max(0, (int)((route_key_score(key) - lo) * vscale)));
+  };
+  // level 0: score buckets; level >= 1: key buckets inside [klo, khi]
+  uint64_t klo = 0, khi = 0;
+  float kscale = 0.f;
+  int level = 0, need = r;
+  auto member_bucket = [&](uint64_t key) -> int {
+    if (level == 0) return vbucket(key);
+    if (key < klo || key > khi) return -1;
+    return min(kBuckets - 1, (int)((float)(key - klo) * kscale));
+  };
+  int bstar = 0, members = 0;
+  if (tid == 0) kred[2 * kRoutedWarps] = ~0ull;  // kth; ordered by the first barrier below
+  for (;;) {
+    for (int i = tid; i < kBuckets; i += kRoutedThreads) hist[i] = 0;
+    if (tid == 0) {
+      misc[0] = 0;
+      misc[1] = 0;
+      misc[2] = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const int bk = member_bucket(keys[i]);
+      if (bk >= 0) atomicAdd(&hist[bk], 1);
+    }
+    __syncthreads();
+    find_boundary_bucket(hist, need, misc);
+    __syncthreads();
+    bstar = misc[0];
+    need -= misc[1];
+    members = hist[bstar];
+    if (members <= kTokRankCap || level >= kTokRefine) break;
+    // key range of the boundary bucket -> the next level's interval
+    uint64_t mn = ~0ull, mx = 0ull;
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const uint64_t key = keys[i];
+      if (member_bucket(key) == bstar) {
+        mn = min(mn, key);
+        mx = max(mx, key);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+      mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
+    if (lane == 0) {
+      kred[2 * warp] = mn;
+      kred[2 * warp + 1] = mx;
+    }
+    __syncthreads();
+    klo = ~0ull;
+    khi = 0ull;
+#pragma unroll
+    for (int w = 0; w < kRoutedWarps; ++w) {
+      klo = min(klo, kred[2 * w]);
+      khi = max(khi, kred[2 * w + 1]);
+    }
+    kscale = (float)kBuckets / ((float)(khi - klo) + 1.0f);
+    ++level;
+    __syncthreads();  // kred and misc are rewritten by the next level
+  }
+  // pairwise ranking of the boundary keys; kth = the need-th largest of them
+  const bool in_scratch = members <= kTokRankCap;
+  if (in_scratch) {
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const uint64_t key = keys[i];
+      if (member_bucket(key) == bstar) {
+        const int slot = atomicAdd(&misc[2], 1);
+        if (slot < kTokRankCap) scratch[slot] = key;
+      }
+    }
+    __syncthreads();
+    const int m = min(members, kTokRankCap);
+    for (int j = tid; j < m; j += kRoutedThreads) {
+      const uint64_t kj = scratch[j];
+      int rank = 0;
+      for (int l = 0; l < m; ++l) rank += scratch[l] > kj;
+      if (rank == need - 1) kred[2 * kRoutedWarps] = kj;
+    }
+  } else {
+    // not reached with distinct keys (each level shrinks the key range by about
+    // kBuckets); ranks the boundary keys against every key
+    for (int i = tid; i < n; i += kRoutedThreads) {
+      const uint64_t ki = keys[i];
+      if (member_bucket(ki) != bstar) continue;
+      int rank = 0;
+      for (int l = 0; l < n; ++l) rank += keys[l] > ki && member_bucket(keys[l]) == bstar;
+      if (rank == need - 1) kred[2 * kRoutedWarps] = ki;
+    }
+  }
+  __syncthreads();
+  const uint64_t kth = kred[2 * kRoutedWarps];
+  const int per = (n + kRoutedThreads - 1) / kRoutedThreads;
+  const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
+  int cnt = 0;
+  for (int i = s0; i < s1; ++i) cnt += keys[i] >= kth;
+  int pos = block_exclusive_scan(cnt, misc + 24);
+  for (int i = s0; i < s1; ++i)
+    if (keys[i] >= kth && pos < r) sel[pos++] = (int)route_key_id(keys[i]);
+}
 
 // Most candidate tokens of the token step over every length up to max_len:
 // C + kcap*C + (last block and tail, < 2C), or every token when nf <= 2 (< 3C).
@@ -217,47 +388,105 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
   // ------------------------------------------------------------- T1 + T2
   const bool keep_all = n_ct <= k_tok;
   if (!keep_all) {
-    const int e0 = (int)((int64_t)n_ct * cr / P), e1 = (int)((int64_t)n_ct * (cr + 1) / P);
-    const int n_rows = e1 - e0;
-    const int nb = (n_rows + 15) / 16;
+    // 16-candidate batches split over the CTAs. C % 16 == 0, so a batch never
+    // straddles two segments (first chunk, a kept chunk, last chunk + tail):
+    // its 16 positions are consecutive and lie in one page, one contiguous run
+    // of K rows that the warp reads with whole-row coalesced loads.
+    const int nbt = (n_ct + 15) / 16;
+    const int bb0 = (int)((int64_t)nbt * cr / P), bb1 = (int)((int64_t)nbt * (cr + 1) / P);
+    const int nb = bb1 - bb0;
+    auto batch_tok = [&](int bi) -> int {  // position of candidate 16 * bi
+      const int e0 = 16 * bi;
+      if (dense) return e0;
+      const int sg = e0 / C;
+      if (sg == 0) return e0;
+      if (sg <= r) return sel[sg - 1] * C + (e0 - sg * C);
+      return tail0 + (e0 - (r + 1) * C);
+    };
     float qv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) qv[j] = qsum[8 * u + j];
-    auto issue = [&](int bi, uint4(&x)[NLD]) {
+    float smin = __int_as_float(0x7f800000), smax = -__int_as_float(0x7f800000);
+    // issue returns the batch's first position; consume takes it back
+    auto issue = [&](int j, uint4(&x)[NLD]) -> int {
+      const int bi = bb0 + j;
+      const int nv = min(16, n_ct - 16 * bi);
+      const int t0 = batch_tok(bi);
+      const uint16_t* src = a.kv.k + (int64_t)tok_row(t0) * D + 8 * u;
+      if (nv == 16) {
 #pragma unroll
-      for (int k = 0; k < NLD; ++k) {
-        const int i = min(16 * bi + RPI * k + rsub, n_rows - 1);
-        x[k] = ldg_stream(a.kv.k + (int64_t)tok_row(cand_tok(e0 + i)) * D + 8 * u);
+        for (int k = 0; k < NLD; ++k) x[k] = ldg_stream(src + (RPI * k + rsub) * D);
+      } else {
+#pragma unroll
+        for (int k = 0; k < NLD; ++k) x[k] = ldg_stream(src + min(RPI * k + rsub, nv - 1) * D);
       }
+      return t0;
     };
-    auto consume = [&](int bi, const uint4(&x)[NLD]) {
+    auto consume = [&](int j, const uint4(&x)[NLD], int t0) {
+      const int bi = bb0 + j;
       float v[NLD];
 #pragma unroll
-      for (int k = 0; k < NLD; ++k) v[k] = dot8(x[k], qv);
+      for (int k = 0; k < NLD; ++k) v[k] = dot8_x2(x[k], qv);
       int idx;
       const float score = butterfly_sum<NLD>(v, lane, idx);
-      const int i = 16 * bi + RPI * idx + rsub;
-      if ((lane & 1) == 0 && i < n_rows) {
-        const int e = e0 + i;
-        const uint64_t key = route_key(score, (uint32_t)cand_tok(e));
-        for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(tkeys, pr)[e] = key;
+      const int i = RPI * idx + rsub;
+      if ((lane & 1) == 0 && i < n_ct - 16 * bi) {
+        const uint64_t key = route_key(score, (uint32_t)(t0 + i));
+        smin = fminf(smin, score);
+        smax = fmaxf(smax, score);
+        if (P == 1) {
+          tkeys[16 * bi + i] = key;
+        } else {
+          for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(tkeys, pr)[16 * bi + i] = key;
+        }
       }
     };
     uint4 xa[NLD], xb[NLD];
-    if (warp < nb) issue(warp, xa);
-    if (warp + kRoutedWarps < nb) issue(warp + kRoutedWarps, xb);
-    for (int bi = warp; bi < nb; bi += 2 * kRoutedWarps) {
-      consume(bi, xa);
-      if (bi + 2 * kRoutedWarps < nb) issue(bi + 2 * kRoutedWarps, xa);
-      if (bi + kRoutedWarps < nb) {
-        consume(bi + kRoutedWarps, xb);
-        if (bi + 3 * kRoutedWarps < nb) issue(bi + 3 * kRoutedWarps, xb);
+    int ta = 0, tb = 0;
+    if (warp < nb) ta = issue(warp, xa);
+    if (warp + kRoutedWarps < nb) tb = issue(warp + kRoutedWarps, xb);
+    for (int j = warp; j < nb; j += 2 * kRoutedWarps) {
+      consume(j, xa, ta);
+      if (j + 2 * kRoutedWarps < nb) ta = issue(j + 2 * kRoutedWarps, xa);
+      if (j + kRoutedWarps < nb) {
+        consume(j + kRoutedWarps, xb, tb);
+        if (j + 3 * kRoutedWarps < nb) tb = issue(j + 3 * kRoutedWarps, xb);
+      }
+    }
+    // score range over the cluster: warp -> CTA -> slot cr of every CTA
+    float* tmm = reinterpret_cast<float*>(hisa_smem + lay.tmm);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      smin = fminf(smin, __shfl_xor_sync(0xFFFFFFFFu, smin, off));
+      smax = fmaxf(smax, __shfl_xor_sync(0xFFFFFFFFu, smax, off));
+    }
+    if (lane == 0) {
+      tmm[2 * kGatherSlots + 2 * warp] = smin;
+      tmm[2 * kGatherSlots + 2 * warp + 1] = smax;
+    }
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int w = 1; w < kRoutedWarps; ++w) {
+        smin = fminf(smin, tmm[2 * kGatherSlots + 2 * w]);
+        smax = fmaxf(smax, tmm[2 * kGatherSlots + 2 * w + 1]);
+      }
+      for (int pr = 0; pr < P; ++pr) {
+        float* dst = cluster.map_shared_rank(tmm, pr);
+        dst[2 * cr] = smin;
+        dst[2 * cr + 1] = smax;
       }
     }
     cluster.sync();
+    float lo = tmm[0], hi = tmm[1];
+    for (int pr = 1; pr < P; ++pr) {
+      lo = fminf(lo, tmm[2 * pr]);
+      hi = fmaxf(hi, tmm[2 * pr + 1]);
+    }
     // top k_tok of the n_ct keys; candidates are in ascending position, so the
     // ordered compaction writes the kept positions ascending
-    select_top_chunks(tkeys, n_ct, k_tok, tsel, hist, misc, scratch, kDecodeScratchKeys);
+    select_top_tokens(tkeys, n_ct, k_tok, lo, hi, tsel, hist, misc, scratch,
+                      reinterpret_cast<uint64_t*>(hisa_smem + lay.kred));
     __syncthreads();
   }
   const int S = keep_all ? n_ct : k_tok;

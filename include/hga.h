@@ -287,7 +287,8 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
  *   out/lse = exact softmax attention over the kept tokens, as hga_attend.
  * idx/n_idx (optional, as hga_decode) receive the kept positions, ascending;
  * idx_stride >= hga_max_hisa_tokens(kv, p, top_tokens). p->group and
- * p->top_groups must be valid as for hga_route but are not used.
+ * p->top_groups must be valid as for hga_route but are not used. p->chunk must
+ * be a multiple of 16 (HGA_ERR_UNSUPPORTED otherwise).
  */
 hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
                            const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,

@@ -106,7 +106,8 @@ def assert_attention_close(gpu: np.ndarray, ref: np.ndarray, what: str) -> None:
 def assert_lse_close(gpu: np.ndarray, ref: np.ndarray, what: str) -> None:
     gpu = np.asarray(gpu, dtype=np.float64)
     both_inf = np.isneginf(gpu) & np.isneginf(ref)
-    err = np.where(both_inf, 0.0, np.abs(gpu - ref))
+    with np.errstate(invalid="ignore"):  # -inf - -inf where both are empty
+        err = np.where(both_inf, 0.0, np.abs(gpu - ref))
     assert (err <= LSE_ATOL + LSE_RTOL * np.where(both_inf, 0.0, np.abs(ref))).all(), f"{what}: lse max err {err.max()}"
 
 
