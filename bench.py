@@ -63,6 +63,7 @@ def decode_bytes(L: int, w=W64) -> int:
 
 DECODE_SOURCES = ("hga_common.cuh", "hga_attention.cuh", "hga_routed.cuh", "hga_decode.cuh")
 PREFILL_SOURCES = ("hga_common.cuh", "hga_tcgen05.cuh", "hga_prefill_attn.cuh")
+HISA_SOURCES = DECODE_SOURCES + ("hga_hisa.cuh",)
 
 
 HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (below the 2304 the two-level route keeps)
@@ -483,7 +484,9 @@ def run_gpu(args, rank: int, world: int, dist):
             "us_per_step": round(hisa_step * 1e3, 2), "queries_per_s": round(B / (hisa_step * 1e-3)),
             "alg_bytes_per_query": hisa_bytes(w.ctx_len),
             "GB_s": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9, 1),
-            "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4)}
+            "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4),
+            "traffic": (lambda t: None if t is None else t * B // 64)(
+                profiled_traffic("hisa_64k_hisa_decode_kernel.md", HISA_SOURCES))}
 
     # host-resident K/V (the pages' placement): 8 of the sequences in pinned, mapped host
     # memory, summaries in HBM; the decode kernel reads only the routed rows over the host link

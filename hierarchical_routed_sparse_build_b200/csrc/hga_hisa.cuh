@@ -15,7 +15,8 @@
 //   R1  chunk scores of candidates 1..nf-2 (as in decode_kernel: 16-row
 //       register batches, halving-butterfly reduction, keys to every CTA)
 //   --  cluster barrier
-//   R2  top-m chunks (bucket select, ascending ids), in every CTA
+//   R2  top-m chunks (select_top_chunks, 256 buckets, ascending ids), in
+//       every CTA
 //   T1  the candidate tokens, [0, C) + the kept chunks' tokens + [(nf-1)C, L)
 //       (every token when nf <= 2), are split over the CTAs in batches of 16
 //       consecutive positions and scored the same way from registers; their
@@ -23,8 +24,8 @@
 //       to every CTA
 //   --  cluster barrier (skipped, with T1 and T2, when the candidates are no
 //       more than the tokens to keep)
-//   T2  top k_tok tokens (select_top_tokens, ascending positions), in every
-//       CTA
+//   T2  top k_tok tokens (select_top_keys on the score range T1 publishes,
+//       ascending positions), in every CTA
 //   A   exact attention over the kept tokens: 16-token tiles split over the
 //       CTAs and round-robin over the warps (hga_attention.cuh), rows staged
 //       in batches of kEntryBatch entries
@@ -34,6 +35,13 @@
 #include "hga_decode.cuh"
 
 namespace hga {
+
+// score-range table in HisaSmem::tmm (floats): token-score range per CTA of
+// the cluster, then per-warp scratch
+constexpr int kTmmTok = 0, kTmmWarp = 2 * kGatherSlots;
+// chunk select: the bit-pattern bucket select of the two-level route with a
+// smaller histogram (measured faster here than 1024 buckets or select_top_keys)
+constexpr int kChunkBuckets = 256;
 
 // Shared-memory carve-up (byte offsets), identical on host and device. The
 // union region holds the chunk keys, the token keys and the select scratch,
@@ -57,7 +65,7 @@ struct HisaSmem {
     hist = o;    o = up16(o + 4 * kBuckets);
     misc = o;    o = up16(o + 4 * 32);
     kred = o;    o = up16(o + 8 * (2 * kRoutedWarps + 2));
-    tmm = o;     o = up16(o + 4 * 2 * (kGatherSlots + kRoutedWarps));
+    tmm = o;     o = up16(o + 4 * (kTmmWarp + 2 * kRoutedWarps));
     rows = o;    o = up16(o + 4 * kEntryBatch);
     tsel = o;    o = up16(o + 4 * k_tok);
     uni = o;
@@ -76,8 +84,50 @@ struct HisaSmem {
   }
 };
 
-constexpr int kTokRankCap = 128;  // boundary keys ranked pairwise in the token select
-constexpr int kTokRefine = 8;     // key-range refinements before the pairwise ranking (7 suffice)
+// Least lo and greatest hi over the CTA's threads, written to slot cr of the
+// table `tab` of every CTA of the cluster (tab[2 cr], tab[2 cr + 1]); the
+// caller's next cluster barrier publishes them. Every thread of the CTA calls it.
+__device__ __forceinline__ void publish_range(float lo, float hi, float* tmm, int tab, cg::cluster_group& cluster,
+                                              int P, int cr) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, off));
+  }
+  if (lane == 0) {
+    tmm[kTmmWarp + 2 * warp] = lo;
+    tmm[kTmmWarp + 2 * warp + 1] = hi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 1; w < kRoutedWarps; ++w) {
+      lo = fminf(lo, tmm[kTmmWarp + 2 * w]);
+      hi = fmaxf(hi, tmm[kTmmWarp + 2 * w + 1]);
+    }
+    for (int pr = 0; pr < P; ++pr) {
+      float* dst = cluster.map_shared_rank(tmm, pr) + tab;
+      dst[2 * cr] = lo;
+      dst[2 * cr + 1] = hi;
+    }
+  }
+}
+
+// The range over the P slots of table `tab` (after the cluster barrier).
+__device__ __forceinline__ void cluster_range(const float* tmm, int tab, int P, float& lo, float& hi) {
+  lo = tmm[tab];
+  hi = tmm[tab + 1];
+  for (int pr = 1; pr < P; ++pr) {
+    lo = fminf(lo, tmm[tab + 2 * pr]);
+    hi = fmaxf(hi, tmm[tab + 2 * pr + 1]);
+  }
+}
+
+constexpr int kTokBuckets = 256;  // select_top_keys histogram (fewer buckets than the bit-pattern select of
+                                  // the two-level route: equal score intervals keep the boundary small)
+constexpr int kTokRankCap = 128;  // boundary keys ranked pairwise in select_top_keys
+constexpr int kTokRefine = 9;     // key-range refinements (each shrinks a 64-bit range ~256x: 8 suffice)
 
 // dot8 with one packed fp32 FMA per bf16 pair: even elements accumulate in .x,
 // odd ones in .y, each rounding exactly like the scalar fmaf chain of dot8.
@@ -97,12 +147,13 @@ __device__ __forceinline__ float route_key_score(uint64_t key) {
 
 // Warp 0 walks the histogram from the top bucket down and finds the bucket
 // holding the need-th key: misc[0] = that bucket, misc[1] = keys above it.
+template <int NB>
 __device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, int* misc) {
   const int lane = threadIdx.x & 31;
   if (threadIdx.x >= 32) return;
-  constexpr int PER = kBuckets / 32;
+  constexpr int PER = NB / 32;
   int tot = 0;
-  for (int k = 0; k < PER; ++k) tot += hist[kBuckets - 1 - PER * lane - k];
+  for (int k = 0; k < PER; ++k) tot += hist[NB - 1 - PER * lane - k];
   int incl = tot;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -113,7 +164,7 @@ __device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, 
   if (excl < need && need <= incl) {
     int acc = excl;
     for (int k = 0; k < PER; ++k) {
-      const int bk = kBuckets - 1 - PER * lane - k;
+      const int bk = NB - 1 - PER * lane - k;
       if (acc + hist[bk] >= need) {
         misc[0] = bk;
         misc[1] = acc;
@@ -127,21 +178,21 @@ __device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, 
 // Top r of n distinct route keys (1 <= r < n), written to sel[] as their ids in
 // the keys' storage order (the token keys are stored in ascending position, so
 // the kept positions come out ascending). lo and hi are the least and greatest
-// score among the keys. The first histogram cuts [lo, hi] into kBuckets equal
+// score among the keys. The first histogram cuts [lo, hi] into kTokBuckets equal
 // score intervals, which for a bell-shaped score distribution leaves a few
 // dozen keys in the bucket holding the r-th key whatever r is (cutting the
 // order-preserving bit pattern instead crowds most keys into the few buckets
 // of the typical magnitude). While that boundary bucket holds more than
-// kTokRankCap keys, its key range is cut again into kBuckets equal intervals
+// kTokRankCap keys, its key range is cut again into kTokBuckets equal intervals
 // of the 64-bit key; the boundary keys are then ranked pairwise. Every bucket
 // map is monotone in the key, so a bucket is a contiguous key range and the
 // kept set equals a full sort's. kred: 2 * kRoutedWarps + 2 words.
-__device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, int r, float lo, float hi, int* sel,
+__device__ __forceinline__ void select_top_keys(const uint64_t* keys, int n, int r, float lo, float hi, int* sel,
                                                   int* hist, int* misc, uint64_t* scratch, uint64_t* kred) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float vscale = hi > lo ? (float)kBuckets / (hi - lo) : 0.f;
+  const float vscale = hi > lo ? (float)kTokBuckets / (hi - lo) : 0.f;
   auto vbucket = [&](uint64_t key) {
-    return min(kBuckets - 1, max(0, (int)((route_key_score(key) - lo) * vscale)));
+    return min(kTokBuckets - 1, max(0, (int)((route_key_score(key) - lo) * vscale)));
   };
   // level 0: score buckets; level >= 1: key buckets inside [klo, khi]
   uint64_t klo = 0, khi = 0;
@@ -150,12 +201,12 @@ __device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, i
   auto member_bucket = [&](uint64_t key) -> int {
     if (level == 0) return vbucket(key);
     if (key < klo || key > khi) return -1;
-    return min(kBuckets - 1, (int)((float)(key - klo) * kscale));
+    return min(kTokBuckets - 1, (int)((float)(key - klo) * kscale));
   };
   int bstar = 0, members = 0;
   if (tid == 0) kred[2 * kRoutedWarps] = ~0ull;  // kth; ordered by the first barrier below
   for (;;) {
-    for (int i = tid; i < kBuckets; i += kRoutedThreads) hist[i] = 0;
+    for (int i = tid; i < kTokBuckets; i += kRoutedThreads) hist[i] = 0;
     if (tid == 0) {
       misc[0] = 0;
       misc[1] = 0;
@@ -167,7 +218,7 @@ __device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, i
       if (bk >= 0) atomicAdd(&hist[bk], 1);
     }
     __syncthreads();
-    find_boundary_bucket(hist, need, misc);
+    find_boundary_bucket<kTokBuckets>(hist, need, misc);
     __syncthreads();
     bstar = misc[0];
     need -= misc[1];
@@ -199,7 +250,7 @@ __device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, i
       klo = min(klo, kred[2 * w]);
       khi = max(khi, kred[2 * w + 1]);
     }
-    kscale = (float)kBuckets / ((float)(khi - klo) + 1.0f);
+    kscale = (float)kTokBuckets / ((float)(khi - klo) + 1.0f);
     ++level;
     __syncthreads();  // kred and misc are rewritten by the next level
   }
@@ -223,7 +274,7 @@ __device__ __forceinline__ void select_top_tokens(const uint64_t* keys, int n, i
     }
   } else {
     // not reached with distinct keys (each level shrinks the key range by about
-    // kBuckets); ranks the boundary keys against every key
+    // kTokBuckets); ranks the boundary keys against every key
     for (int i = tid; i < n; i += kRoutedThreads) {
       const uint64_t ki = keys[i];
       if (member_bucket(ki) != bstar) continue;
@@ -277,6 +328,8 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
   int* misc = reinterpret_cast<int*>(hisa_smem + lay.misc);
   uint32_t* rows = reinterpret_cast<uint32_t*>(hisa_smem + lay.rows);
   int* tsel = reinterpret_cast<int*>(hisa_smem + lay.tsel);
+  float* tmm = reinterpret_cast<float*>(hisa_smem + lay.tmm);
+  uint64_t* kred = reinterpret_cast<uint64_t*>(hisa_smem + lay.kred);
   uint64_t* ckeys = reinterpret_cast<uint64_t*>(hisa_smem + lay.ckeys);
   uint64_t* tkeys = reinterpret_cast<uint64_t*>(hisa_smem + lay.tkeys);
   uint64_t* scratch = reinterpret_cast<uint64_t*>(hisa_smem + lay.scratch);
@@ -333,7 +386,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
     auto consume = [&](int bi, const uint4(&x)[NLD]) {
       float v[NLD];
 #pragma unroll
-      for (int k = 0; k < NLD; ++k) v[k] = dot8(x[k], qv);
+      for (int k = 0; k < NLD; ++k) v[k] = dot8_x2(x[k], qv);
       int idx;
       const float score = butterfly_sum<NLD>(v, lane, idx);
       const int i = 16 * bi + RPI * idx + rsub;
@@ -371,7 +424,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
 
   // ------------------------------------------------------------------ R2
   if (select_needed) {
-    select_top_chunks(ckeys, n_cand, r, sel, hist, misc, scratch, kDecodeScratchKeys);
+    select_top_chunks<kChunkBuckets>(ckeys, n_cand, r, sel, hist, misc, scratch, kDecodeScratchKeys);
   } else {
     for (int i = tid; i < r; i += kRoutedThreads) sel[i] = i + 1;
   }
@@ -453,40 +506,13 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
         if (j + 3 * kRoutedWarps < nb) tb = issue(j + 3 * kRoutedWarps, xb);
       }
     }
-    // score range over the cluster: warp -> CTA -> slot cr of every CTA
-    float* tmm = reinterpret_cast<float*>(hisa_smem + lay.tmm);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      smin = fminf(smin, __shfl_xor_sync(0xFFFFFFFFu, smin, off));
-      smax = fmaxf(smax, __shfl_xor_sync(0xFFFFFFFFu, smax, off));
-    }
-    if (lane == 0) {
-      tmm[2 * kGatherSlots + 2 * warp] = smin;
-      tmm[2 * kGatherSlots + 2 * warp + 1] = smax;
-    }
-    __syncthreads();
-    if (tid == 0) {
-#pragma unroll
-      for (int w = 1; w < kRoutedWarps; ++w) {
-        smin = fminf(smin, tmm[2 * kGatherSlots + 2 * w]);
-        smax = fmaxf(smax, tmm[2 * kGatherSlots + 2 * w + 1]);
-      }
-      for (int pr = 0; pr < P; ++pr) {
-        float* dst = cluster.map_shared_rank(tmm, pr);
-        dst[2 * cr] = smin;
-        dst[2 * cr + 1] = smax;
-      }
-    }
+    publish_range(smin, smax, tmm, kTmmTok, cluster, P, cr);
     cluster.sync();
-    float lo = tmm[0], hi = tmm[1];
-    for (int pr = 1; pr < P; ++pr) {
-      lo = fminf(lo, tmm[2 * pr]);
-      hi = fmaxf(hi, tmm[2 * pr + 1]);
-    }
+    float lo, hi;
+    cluster_range(tmm, kTmmTok, P, lo, hi);
     // top k_tok of the n_ct keys; candidates are in ascending position, so the
     // ordered compaction writes the kept positions ascending
-    select_top_tokens(tkeys, n_ct, k_tok, lo, hi, tsel, hist, misc, scratch,
-                      reinterpret_cast<uint64_t*>(hisa_smem + lay.kred));
+    select_top_keys(tkeys, n_ct, k_tok, lo, hi, tsel, hist, misc, scratch, kred);
     __syncthreads();
   }
   const int S = keep_all ? n_ct : k_tok;

@@ -201,6 +201,7 @@ __device__ __forceinline__ void stream_rows(uint4* stage, int stage_rows, int n_
 //   3. ordered compaction of keys >= K_r (candidate order = ascending ids).
 // scratch must hold scratch_cap keys; if b* holds more, ranking falls back to
 // scanning all n keys (correct, slower; only for near-constant scores).
+template <int NB = kBuckets>
 __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, int r, int* sel,
                                                   int* hist, int* misc, uint64_t* scratch,
                                                   int scratch_cap) {
@@ -220,7 +221,7 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
     misc[8 + warp] = (int)lo;
     misc[16 + warp] = (int)hi;
   }
-  for (int i = tid; i < kBuckets; i += kRoutedThreads) hist[i] = 0;
+  for (int i = tid; i < NB; i += kRoutedThreads) hist[i] = 0;
   if (tid == 0) misc[2] = 0;
   __syncthreads();
   lo = 0xFFFFFFFFu;
@@ -230,14 +231,14 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
     lo = min(lo, (uint32_t)misc[8 + w]);
     hi = max(hi, (uint32_t)misc[16 + w]);
   }
-  const float scale = (float)kBuckets / ((float)(hi - lo) + 1.0f);
-  auto bucket = [&](uint32_t u) { return min(kBuckets - 1, (int)((float)(u - lo) * scale)); };
+  const float scale = (float)NB / ((float)(hi - lo) + 1.0f);
+  auto bucket = [&](uint32_t u) { return min(NB - 1, (int)((float)(u - lo) * scale)); };
   for (int i = tid; i < n; i += kRoutedThreads) atomicAdd(&hist[bucket((uint32_t)(keys[i] >> 32))], 1);
   __syncthreads();
   if (warp == 0) {
-    constexpr int PER = kBuckets / 32;
+    constexpr int PER = NB / 32;
     int tot = 0;
-    for (int k = 0; k < PER; ++k) tot += hist[kBuckets - 1 - PER * lane - k];
+    for (int k = 0; k < PER; ++k) tot += hist[NB - 1 - PER * lane - k];
     int incl = tot;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -248,7 +249,7 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
     if (excl < r && r <= incl) {
       int acc = excl;
       for (int k = 0; k < PER; ++k) {
-        const int b = kBuckets - 1 - PER * lane - k;
+        const int b = NB - 1 - PER * lane - k;
         if (acc + hist[b] >= r) {
           misc[0] = b;
           misc[1] = acc;

@@ -122,3 +122,38 @@ def test_hisa_decode_64k_sampled(hga):
     inp = synth.decode_inputs(w, lengths=[w.ctx_len] * 2)
     exact, n = run_hisa(hga, w, inp, m=32, k_tok=2048, units=[(0, 0), (0, 3), (1, 1)])
     assert exact >= n - 1
+
+
+@pytest.mark.parametrize("ctas", [0, 3])
+def test_hisa_ties_take_lower_positions(hga, ctas):
+    # every key equal: all chunk summaries and all token scores tie, so the kept
+    # set is the first k_tok candidates by position (the select's refinement path)
+    w = synth.Workload("hisa_ties", 1, 32, 4, 128, 9000, 128, 16, 8, 2, -1, 47)
+    inp = synth.decode_inputs(w, lengths=[9000, 6100], max_len=9088)
+    inp.k[:] = inp.k[:, :, :1, :]
+    hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, ctas)
+    try:
+        from hierarchical_routed_sparse_build_b200.runtime import RoutedCache
+        c = RoutedCache(inp.k, inp.v, inp.seq_lens, chunk=128, group=16, top_chunks=8, top_groups=2, n_q_heads=32)
+        c.build_summaries()
+        out, _, idx, n_idx = c.decode_hisa(c.q_tensor(inp.q), 700, want_idx=True)
+        assert hga.hga_get_device_error()[0] == 0
+    finally:
+        hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
+    for b, L in enumerate(inp.seq_lens):
+        assert oracle.hisa_candidates(int(L), 128, 8) > 700
+        for h in range(4):
+            K = inp.k[b, h, :L]
+            cs, _ = oracle.summaries(K, 128, 16)
+            ref = oracle.hisa_route(inp.q[b, h * 8:(h + 1) * 8], cs, K, int(L), 128, 8, 700)
+            assert np.array_equal(ref, np.arange(700))  # chunks 1..8 win their ties
+            assert n_idx[b, h].item() == 700
+            assert np.array_equal(idx[b, h, :700].cpu().numpy(), ref), f"ties b{b} h{h}"
+
+
+def test_hisa_many_blocks(hga):
+    # 64 kept chunks of 126 at 16K: 8448 candidate tokens in shared memory
+    w = synth.DECODE_16K
+    inp = synth.decode_inputs(w, lengths=[w.ctx_len] * 2)
+    exact, n = run_hisa(hga, w, inp, m=64, k_tok=3000, units=[(0, 0), (0, 2), (1, 3)])
+    assert exact >= n - 1
