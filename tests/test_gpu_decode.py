@@ -180,6 +180,36 @@ def test_cluster_sizes_agree(hga, ctas, kernel):
     assert exact >= n - 1
 
 
+def test_one_cta_per_head_ragged_and_paged(hga):
+    # one CTA per (sequence, KV head), the automatic choice above 148 units, on
+    # ragged lengths (dense units included), then the same sequences in shuffled
+    # pages: the paged decode must equal the contiguous one bit for bit
+    w = synth.Workload("onecta", 1, 32, 4, 128, 0, 128, 16, 6, 2, -1, 61)
+    lens = [0, 1, 200, 383, 384, 385, 700, 1024, 2049, 3000, 4095, 4096]
+    inp = synth.decode_inputs(w, lengths=lens, max_len=4096)
+    hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 1)
+    try:
+        exact, n = run_and_check(hga, w, inp, check_summaries=False)
+        assert exact >= n - 1
+        B, per = len(lens), 4096 // 128
+        table = np.random.default_rng(13).permutation(B * per).astype(np.int32).reshape(B, per)
+        kpool = np.zeros((B * per, 4, 128, 128), dtype=np.uint16)
+        vpool = np.zeros_like(kpool)
+        for b in range(B):
+            kpool[table[b]] = inp.k[b].reshape(4, per, 128, 128).transpose(1, 0, 2, 3)
+            vpool[table[b]] = inp.v[b].reshape(4, per, 128, 128).transpose(1, 0, 2, 3)
+        c = cache_for(hga, w, kpool, vpool, inp.seq_lens, page_table=table)
+        out_p, lse_p, idx_p, n_p = c.decode(c.q_tensor(inp.q), want_idx=True)
+        no_device_error(hga)
+        c2 = cache_for(hga, w, inp.k, inp.v, inp.seq_lens)
+        out_c, lse_c, idx_c, n_c = c2.decode(c2.q_tensor(inp.q), want_idx=True)
+        no_device_error(hga)
+        assert torch.equal(n_p, n_c) and torch.equal(idx_p, idx_c)
+        assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+    finally:
+        hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
+
+
 @pytest.mark.parametrize("group,chunk,top_groups", [(8, 128, 4), (32, 128, 2), (16, 64, 4), (16, 256, 3)])
 def test_group_sizes(hga, group, chunk, top_groups):
     # g = 8 runs the phase-by-phase kernel (a 16-token tile spans two groups);
