@@ -121,3 +121,70 @@ def test_launch_option_validation():
     with pytest.raises(hga.HgaError):
         hga.hga_set_launch_option(7, 1)
     hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
+
+
+def raw_hisa(kv, p, top_tokens=2048, q=FAKE, cs=FAKE, out=FAKE, idx=None, stride=0, n_idx=None, hq=32):
+    return hga._lib.hga_decode_hisa(q, hq, ctypes.byref(kv), cs, ctypes.byref(p), top_tokens, out, None, idx,
+                                    stride, n_idx, None)
+
+
+def test_hisa_rejects_bad_arguments_on_host():
+    kv, p = kv_desc(), params()
+    assert raw_hisa(kv, p, top_tokens=0) == INVALID
+    assert raw_hisa(kv, p, q=0) == INVALID
+    assert raw_hisa(kv, p, cs=0) == INVALID
+    assert raw_hisa(kv, p, cs=FAKE + 8) == INVALID
+    assert raw_hisa(kv, p, out=0) == INVALID
+    assert raw_hisa(kv, p, idx=FAKE, stride=4096, n_idx=None) == INVALID      # idx without n_idx
+    assert raw_hisa(kv, p, idx=FAKE, stride=100, n_idx=FAKE) == INVALID       # stride below the bound
+    assert raw_hisa(kv, params(chunk=24, group=8, top_groups=2)) == UNSUPPORTED  # 16-token batches span chunks
+    assert raw_hisa(kv, p, hq=48) == UNSUPPORTED                              # 12 query heads per KV head
+    assert raw_hisa(kv_desc(head_dim=96), p) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("max_len,C,m,k_tok", [
+    (65536, 128, 32, 2048), (16384, 128, 64, 3000), (4096, 64, 8, 700), (300, 64, 4, 100),
+    (65536 + 77, 128, 32, 100000), (9088, 128, 8, 1024), (383, 128, 2, 5000), (384, 128, 2, 5000),
+])
+def test_max_hisa_tokens_bounds_every_length(max_len, C, m, k_tok):
+    kv = kv_desc(max_len=max_len, head_dim=64)
+    n = hga._lib.hga_max_hisa_tokens(ctypes.byref(kv), ctypes.byref(params(chunk=C, group=16, top_chunks=m,
+                                                                           top_groups=2)), k_tok)
+    want = max(min(k_tok, oracle.hisa_candidates(L, C, m)) for L in range(1, max_len + 1))
+    assert n == want
+
+
+def test_append_rejects_bad_arguments_on_host():
+    kv, p = kv_desc(), params()
+    L = hga._lib
+    other_lens = FAKE + 0x100  # not the descriptor's seq_lens
+    assert L.hga_append(ctypes.byref(kv), other_lens, FAKE, FAKE, ctypes.byref(p), FAKE, FAKE, None) == INVALID
+    assert L.hga_append(ctypes.byref(kv), FAKE, FAKE + 8, FAKE, ctypes.byref(p), FAKE, FAKE, None) == INVALID
+    assert L.hga_append(ctypes.byref(kv), FAKE, FAKE, FAKE, ctypes.byref(p), None, FAKE, None) == INVALID
+    assert L.hga_append(ctypes.byref(kv_desc(v=0)), FAKE, FAKE, FAKE, ctypes.byref(p), FAKE, FAKE, None) == INVALID
+
+
+def raw_prefill(kv, p, n_queries=2048, block=64, cache_len=63488, hq=32, out=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return hga._lib.hga_prefill(FAKE, hq, n_queries, block, ctypes.byref(kv), cache_len, FAKE, FAKE,
+                                ctypes.byref(p), out, ws, ws_bytes, None)
+
+
+def test_prefill_rejects_bad_arguments_on_host():
+    kv1, p = kv_desc(batch=1), params()
+    assert raw_prefill(kv1, p, cache_len=65536 - 2047) == INVALID           # past max_len
+    assert raw_prefill(kv1, p, n_queries=0) == INVALID
+    assert raw_prefill(kv1, p, cache_len=-1) == INVALID
+    assert raw_prefill(kv1, p, out=0) == INVALID
+    assert raw_prefill(kv1, p, ws=0) == INVALID
+    assert raw_prefill(kv1, p, ws_bytes=16) == INVALID                      # workspace too small
+    assert raw_prefill(kv_desc(batch=2), p) == UNSUPPORTED                 # one sequence per call
+    assert raw_prefill(kv1, p, block=32) == UNSUPPORTED
+    assert raw_prefill(kv1, p, n_queries=2000) == UNSUPPORTED               # not a multiple of the block
+    assert raw_prefill(kv_desc(batch=1, head_dim=64), p) == UNSUPPORTED
+
+
+def test_prefill_workspace_holds_the_lists():
+    kv1, p = kv_desc(batch=1), params()
+    need = hga._lib.hga_prefill_workspace_size(ctypes.byref(kv1), 32, 2048, 64, 63488, ctypes.byref(p))
+    stride = oracle.max_routed(63488, 128, 16, 32, 4)
+    assert need >= 32 * 4 * (stride + 1) * 4
