@@ -288,7 +288,11 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
  * idx/n_idx (optional, as hga_decode) receive the kept positions, ascending;
  * idx_stride >= hga_max_hisa_tokens(kv, p, top_tokens). p->group and
  * p->top_groups must be valid as for hga_route but are not used. p->chunk must
- * be a multiple of 16 (HGA_ERR_UNSUPPORTED otherwise).
+ * be a multiple of 16, and the token keys of the most candidates at any length
+ * ((min(top_chunks, max_len / chunk - 2) + 3) * chunk of them, 8 bytes each)
+ * plus the kept list (4 bytes per kept token) must fit one CTA's 227 KB of
+ * shared memory with the rest of its state (about 37 KB at head_dim 128);
+ * HGA_ERR_UNSUPPORTED otherwise.
  */
 hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
                            const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,

@@ -188,3 +188,9 @@ def test_prefill_workspace_holds_the_lists():
     need = hga._lib.hga_prefill_workspace_size(ctypes.byref(kv1), 32, 2048, 64, 63488, ctypes.byref(p))
     stride = oracle.max_routed(63488, 128, 16, 32, 4)
     assert need >= 32 * 4 * (stride + 1) * 4
+
+
+def test_hisa_rejects_candidate_sets_beyond_shared_memory():
+    # 64K context, top 510 chunks: (510 + 3) * 128 candidate keys of 8 bytes do not fit one CTA
+    kv, p = kv_desc(), params(top_chunks=510)
+    assert raw_hisa(kv, p) == UNSUPPORTED
