@@ -194,3 +194,19 @@ def test_hisa_rejects_candidate_sets_beyond_shared_memory():
     # 64K context, top 510 chunks: (510 + 3) * 128 candidate keys of 8 bytes do not fit one CTA
     kv, p = kv_desc(), params(top_chunks=510)
     assert raw_hisa(kv, p) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("cache_len,n_queries,C,g,k,G", [
+    (63488, 2048, 128, 16, 32, 4), (1000, 512, 128, 16, 4, 2), (0, 256, 128, 16, 8, 4),
+    (4000, 1024, 64, 16, 8, 2), (383, 128, 128, 16, 2, 1),
+])
+def test_prefill_workspace_sizes_hold_the_longest_list(cache_len, n_queries, C, g, k, G):
+    kv1 = kv_desc(batch=1, max_len=cache_len + n_queries)
+    p = params(chunk=C, group=g, top_chunks=k, top_groups=G)
+    units = (n_queries // 64) * 4
+    plain = hga._lib.hga_prefill_workspace_size(ctypes.byref(kv1), 32, n_queries, 64, cache_len, ctypes.byref(p))
+    assert plain == units * (oracle.max_routed(cache_len, C, g, k, G) + 1) * 4
+    grow = hga._lib.hga_prefill_growing_workspace_size(ctypes.byref(kv1), 32, n_queries, 64, cache_len,
+                                                       ctypes.byref(p))
+    longest = max(oracle.max_routed(cache_len + 64 * b, C, g, k, G) for b in range(n_queries // 64))
+    assert grow == units * (longest + 1) * 4
