@@ -322,6 +322,28 @@ def oracle_queries_per_s(inp, w, seconds: float, max_threads: int | None = None)
                                   f"({queries:.0f} queries) in {dt:.1f} s, summaries prebuilt"
 
 
+def cpu_model() -> str:
+    """The host CPU's model string (Linux /proc/cpuinfo), for the baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline_record(inp, w, seconds: float, single_seconds: float = 3.0) -> dict:
+    """The oracle on every host thread (the baseline value) and, on a short sample, on one thread."""
+    v, cores, sample = oracle_queries_per_s(inp, w, seconds)
+    v1, _, sample1 = oracle_queries_per_s(inp, w, single_seconds, max_threads=1)
+    return {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model(), "single_thread": {"value": round(v1, 3), "unit": UNIT, "sample": sample1}}
+
+
 # --------------------------------------------------------------------------- ranks
 
 
@@ -601,7 +623,7 @@ def main():
             "config": {"workload": "decode_64k (same shapes and routing as our arm), CPU oracle on 8 sequences",
                        "batch_per_gpu": 8, "ctx_len": w.ctx_len},
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }), flush=True)
         return
@@ -617,9 +639,7 @@ def main():
         res, inp, w = run_gpu(args, rank, world, dist)
         if rank == 0:
             if not args.no_cpu_baseline and world == 1:
-                v, cores, sample = oracle_queries_per_s(inp, w, args.cpu_seconds)
-                res["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                                       "sample": sample}
+                res["cpu_baseline"] = cpu_baseline_record(inp, w, args.cpu_seconds)
             print(json.dumps(res), flush=True)
     finally:
         if dist is not None:
