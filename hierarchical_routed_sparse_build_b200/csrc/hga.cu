@@ -646,14 +646,16 @@ hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, c
   a.hq = n_q_heads;
   a.R = n_q_heads / kv->n_kv_heads;
   routing_args(a, kv, p);
-  a.k_tok = top_tokens;
+  // never more than the most candidates at any length: a larger top_tokens keeps every candidate
+  // either way, and this bounds the shared-memory list
+  a.k_tok = hisa_max_routed(kv, p, top_tokens);
   a.scale_log2 = scale_log2(p, kv->head_dim);
   a.out = out;
   a.lse = lse;
   a.idx_out = idx;
   a.n_idx_out = n_idx;
   a.idx_stride = idx ? idx_stride : 0;
-  const int smem = HisaSmem(kv->head_dim, a.n_pad, a.kcap, hisa_tok_pad(p->chunk, a.kcap), top_tokens).total;
+  const int smem = HisaSmem(kv->head_dim, a.n_pad, a.kcap, hisa_tok_pad(p->chunk, a.kcap), a.k_tok).total;
   if (smem > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
   const int units = kv->batch * kv->n_kv_heads;
   const int P = pick_cluster(units);

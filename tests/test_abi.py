@@ -210,3 +210,11 @@ def test_prefill_workspace_sizes_hold_the_longest_list(cache_len, n_queries, C, 
                                                        ctypes.byref(p))
     longest = max(oracle.max_routed(cache_len + 64 * b, C, g, k, G) for b in range(n_queries // 64))
     assert grow == units * (longest + 1) * 4
+
+
+def test_hisa_kept_list_is_bounded_by_the_candidates():
+    # a top_tokens above every length's candidate count keeps every candidate; the
+    # kept list (and the shared memory it takes) is bounded by the candidates
+    kv, p = kv_desc(), params()
+    assert hga._lib.hga_max_hisa_tokens(ctypes.byref(kv), ctypes.byref(p), 10_000_000) == \
+        max(oracle.hisa_candidates(L, 128, 32) for L in range(65536 - 256, 65537))
