@@ -366,6 +366,39 @@ def weak_scaling_rate(units_per_rank: int, world: int, steps: int, total_ms: flo
 # --------------------------------------------------------------------------- GPU arm
 
 
+def run_paged_batch(hga, RoutedCache, dev, timed, n: int) -> dict:
+    """The batched decode on a paged pool: 16 ragged sequences of 4K-64K tokens (seeded lengths), page =
+    chunk = 128 tokens, shuffled page table, L2 flushed between steps. A failure here is recorded in the
+    object rather than ending the run."""
+    try:
+        wp = synth.BATCHED_PAGED
+        pin = synth.paged_inputs(wp)
+        pc = RoutedCache(pin.k_pool, pin.v_pool, pin.seq_lens, chunk=wp.chunk, group=wp.group,
+                         top_chunks=wp.top_chunks, top_groups=wp.top_groups, n_q_heads=wp.n_q_heads,
+                         page_table=pin.page_table, device=dev)
+        pc.build_summaries()
+        pq = pc.q_tensor(pin.q)
+        pout, plse = pc.out_buffers()
+        for _ in range(3):
+            pc.decode(pq, pout, plse)
+        times = timed(n, lambda: pc.decode(pq, pout, plse))
+        st, bits = hga.hga_get_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error bits {bits}")
+        step_ms = statistics.median(times)
+        lens = [int(x) for x in pin.seq_lens]
+        nbytes = sum(decode_bytes(L) for L in lens)
+        hbm, _ = peaks()
+        return {"what": "hga_decode on a paged pool: 16 sequences of seeded lengths in [4096, 65536], page = chunk = "
+                        "128 tokens, shuffled page table",
+                "lengths": {"min": min(lens), "max": max(lens), "total": sum(lens)},
+                "us_per_step": round(step_ms * 1e3, 2), "queries_per_s": round(len(lens) / (step_ms * 1e-3)),
+                "alg_bytes_per_step": nbytes, "GB_s": round(nbytes / (step_ms * 1e-3) / 1e9, 1),
+                "frac_hbm": round(nbytes / (step_ms * 1e-3) / 1e9 / hbm, 4)}
+    except Exception as exc:  # recorded, so that the rest of the line is still printed
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
 def run_gpu(args, rank: int, world: int, dist):
     import torch
 
@@ -544,6 +577,7 @@ def run_gpu(args, rank: int, world: int, dist):
     srt = sorted(times)
     pct = lambda p: srt[min(len(srt) - 1, int(round(p / 100 * (len(srt) - 1))))]
     prefill = None if args.no_prefill else run_prefill(dev, max(5, args.steps // 10), args.warmup)
+    paged = run_paged_batch(hga, RoutedCache, dev, timed, max(10, args.steps // 2))
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -572,6 +606,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "decode_loop_graph": decode_loop,
         "host_resident_kv": host_kv,
         "block_then_token": hisa,
+        "paged_batch": paged,
         "prefill": prefill,
     }
     return res, inp, w
