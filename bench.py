@@ -366,6 +366,27 @@ def weak_scaling_rate(units_per_rank: int, world: int, steps: int, total_ms: flo
 # --------------------------------------------------------------------------- GPU arm
 
 
+def run_summaries(hga, cache, timed, B: int, n: int = 5) -> dict:
+    """Summary build over the whole cache (amortised over decode steps): K read once, chunk and group
+    means written. Recorded as an error object if it fails."""
+    try:
+        times = timed(n, cache.build_summaries)
+        st, bits = hga.hga_get_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error bits {bits}")
+        ms = statistics.median(times)
+        w = W64
+        nf = w.ctx_len // w.chunk
+        per_head = w.ctx_len * w.head_dim * 2 + nf * w.head_dim * 2 * (1 + w.chunk // w.group)
+        nbytes = B * w.n_kv_heads * per_head
+        hbm, _ = peaks()
+        return {"what": f"hga_build_summaries over {B} x 64K sequences (K read once; chunk and group means "
+                        "written)", "us_per_call": round(ms * 1e3, 1), "alg_bytes": nbytes,
+                "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+    except Exception as exc:  # recorded, so that the rest of the line is still printed
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
 def run_paged_batch(hga, RoutedCache, dev, timed, n: int) -> dict:
     """The batched decode on a paged pool: 16 ragged sequences of 4K-64K tokens (seeded lengths), page =
     chunk = 128 tokens, shuffled page table, L2 flushed between steps. A failure here is recorded in the
@@ -578,6 +599,7 @@ def run_gpu(args, rank: int, world: int, dist):
     pct = lambda p: srt[min(len(srt) - 1, int(round(p / 100 * (len(srt) - 1))))]
     prefill = None if args.no_prefill else run_prefill(dev, max(5, args.steps // 10), args.warmup)
     paged = run_paged_batch(hga, RoutedCache, dev, timed, max(10, args.steps // 2))
+    summaries = run_summaries(hga, cache, timed, B)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -607,6 +629,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "host_resident_kv": host_kv,
         "block_then_token": hisa,
         "paged_batch": paged,
+        "summaries": summaries,
         "prefill": prefill,
     }
     return res, inp, w
