@@ -136,7 +136,6 @@ def run_prefill(dev, steps: int, warmup: int):
     import torch
 
     import hierarchical_routed_sparse_build_b200 as hga
-    import oracle
 
     w = synth.PREFILL_64K
     inp = synth.prefill_inputs(w)
@@ -152,8 +151,9 @@ def run_prefill(dev, steps: int, warmup: int):
     hga.hga_build_summaries(kv, p, cs, gs)
     wsb = hga.hga_prefill_workspace_size(kv, w.n_q_heads, T, w.block, L0, p)
     ws = torch.zeros(wsb // 4, dtype=torch.int32, device=dev)
-    stride = oracle.max_routed(L0, w.chunk, w.group, w.top_chunks, w.top_groups)
     nb = T // w.block
+    # the workspace holds [blocks][KV heads][stride] routed positions, then one count per list
+    stride = wsb // (4 * nb * w.n_kv_heads) - 1
     idx = ws[: nb * w.n_kv_heads * stride].view(nb, w.n_kv_heads, stride)
     n_idx = ws[nb * w.n_kv_heads * stride: nb * w.n_kv_heads * (stride + 1)].view(nb, w.n_kv_heads)
     out = torch.empty((T, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)

@@ -27,7 +27,7 @@ __all__ = [
     "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
     "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer", "hga_decode_hisa", "hga_max_hisa_tokens",
     "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
-    "HGA_OPT_PREFILL_KERNEL", "STATUS_NAMES",
+    "HGA_OPT_TEST_EXPIRE_PREFILL_WAIT", "STATUS_NAMES",
     "EXPORTED",
 ]
 
@@ -37,7 +37,7 @@ _LIB_PATH = os.path.join(_HERE, "libhga.so")
 HGA_OK = 0
 HGA_OPT_CTAS_PER_HEAD = 1
 HGA_OPT_DECODE_KERNEL = 2
-HGA_OPT_PREFILL_KERNEL = 3
+HGA_OPT_TEST_EXPIRE_PREFILL_WAIT = 4
 STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_UNSUPPORTED", 3: "HGA_ERR_CUDA",
                 4: "HGA_ERR_DEVICE_FAULT", 5: "HGA_ERR_TIMEOUT"}
 EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens", "hga_route",

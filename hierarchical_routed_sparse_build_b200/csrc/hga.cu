@@ -17,7 +17,6 @@
 #include "hga_decode.cuh"
 #include "hga_hisa.cuh"
 #include "hga_prefill_attn.cuh"
-#include "hga_prefill_attn2.cuh"
 #include "hga_prefill_route.cuh"
 #include "hga_routed.cuh"
 #include "hga_summaries.cuh"
@@ -27,7 +26,7 @@ namespace {
 
 std::atomic<int> g_ctas_per_head{0};
 std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 phase-by-phase, 2 fused
-std::atomic<int> g_prefill_kernel{0};  // 0 automatic (one Q tile per CTA), 1 one tile, 2 two tiles
+std::atomic<int> g_fail_at_tile{-1};  // test hook of the prefill attention kernel (-1: off)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -340,6 +339,7 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
   a.scale_log2 = scale_log2(p, kv->head_dim);
   a.out = out;
   a.growing = growing ? 1 : 0;
+  a.fail_at_tile = g_fail_at_tile.load();
   static std::atomic<bool> configured[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
@@ -355,18 +355,6 @@ hga_status launch_prefill_attend(const void* q, int32_t n_q_heads, int32_t n_que
     configured[dev].store(true);
   }
   const int m_tiles = a.R * block / kPfRows;
-  if (m_tiles % 2 == 0 && g_prefill_kernel.load() == 2) {
-    static std::atomic<bool> configured2[kMaxDevices];
-    if (!configured2[dev].load()) {
-      if (cudaFuncSetAttribute(prefill_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Prefill2Smem::kTotal) != cudaSuccess)
-        return HGA_ERR_CUDA;
-      configured2[dev].store(true);
-    }
-    const int grid2 = (n_queries / block) * kv->n_kv_heads * (m_tiles / 2);
-    prefill_attn2_kernel<<<grid2, kPf2Threads, Prefill2Smem::kTotal, stream>>>(a);
-    return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
-  }
   const int grid = (n_queries / block) * kv->n_kv_heads * m_tiles;
   prefill_attn_kernel<<<grid, kPfThreads, PrefillSmem::kTotal, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
@@ -817,9 +805,9 @@ hga_status hga_set_launch_option(int32_t option, int32_t value) {
     g_decode_kernel.store(value);
     return HGA_OK;
   }
-  if (option == HGA_OPT_PREFILL_KERNEL) {
-    if (value < 0 || value > 2) return HGA_ERR_INVALID_ARG;
-    g_prefill_kernel.store(value);
+  if (option == HGA_OPT_TEST_EXPIRE_PREFILL_WAIT) {
+    if (value < 0) return HGA_ERR_INVALID_ARG;
+    g_fail_at_tile.store(value - 1);
     return HGA_OK;
   }
   return HGA_ERR_INVALID_ARG;

@@ -18,6 +18,14 @@
 // K/V tiles are gathered row by row with cp.async (double-buffered stages), since
 // the routed keys are arbitrary runs of rows. One thread issues the MMAs and
 // commits them to mbarriers; every wait is bounded and reports kErrTimeout.
+//
+// Exit after an expired wait: the CTA stops issuing MMAs and copies, then every
+// thread waits (bounded) for the last S and the last PV it committed, so that no
+// tcgen05.mma is outstanding when tensor memory is released. Only if one of
+// those final waits also expires (an MMA that never completes, which no input
+// can cause) does the CTA leave without deallocating, rather than free columns
+// an MMA may still write; the timeout is reported either way and no output row
+// of the CTA is written.
 // The softmax keeps a reference maximum per row and rescales the TMEM
 // accumulator only when a new maximum exceeds it by more than 2^8 (exact: the
 // final division uses the same reference).
@@ -46,6 +54,7 @@ struct PrefillAttnArgs {
   int idx_stride;
   float scale_log2;
   float* out;          // [T][Hq][128]
+  int fail_at_tile;    // test hook: >= 0 makes key tile j's S wait report expiry after it has completed
 };
 
 // Dynamic shared memory, offsets from a 1024-byte aligned base.
@@ -170,6 +179,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
   float m_ref = -INFINITY, l_sum = 0.f;
   const float sl = a.scale_log2;
   bool ok = true;
+  // index of the last S and PV committed (every thread follows the same control
+  // flow, so all agree); the exit waits for both before releasing tensor memory
+  int last_s = -1, last_o = -1;
 
   for (int j = 0; j < n_tiles; ++j) {
     const int st = j & 1;
@@ -178,6 +190,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     __syncthreads();
     if (*abort_flag) break;
     // S = Q K_j^T
+    last_s = j;
     if (tid == 0) {
       tc_fence_after();
       const uint32_t aK = smem_u32(smem + PrefillSmem::kK + st * 16384);
@@ -191,10 +204,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     }
     // stage j-1 is free once PV_{j-1} has completed; then prefetch tile j+1 into it
     if (j >= 1 && !mbar_wait_bounded(bar_o, (uint32_t)((j - 1) & 1))) ok = false;
-    if (j + 1 < n_tiles) issue_tile(j + 1, next_tok, st ^ 1);
+    if (j + 1 < n_tiles && ok) issue_tile(j + 1, next_tok, st ^ 1);
     cp_async_commit();
     if (j + 2 < n_tiles) tile_tokens(j + 2, next_tok);  // list entries of the tile after next
-    if (!mbar_wait_bounded(bar_s, (uint32_t)(j & 1))) ok = false;
+    if (!mbar_wait_bounded(bar_s, (uint32_t)(j & 1)) || j == a.fail_at_tile) ok = false;
     tc_fence_after();
 
     // softmax of this thread's row; only tiles reaching past the routed cache
@@ -228,7 +241,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
       m_ref = tmax;
       l_sum *= alpha;
     }
-    if (j >= 1 && __any_sync(0xFFFFFFFFu, need && alpha != 1.f)) {
+    // (warp-uniform condition; skipped once a wait has expired, as PV_{j-1} may
+    // then still be writing the accumulator)
+    if (j >= 1 && __any_sync(0xFFFFFFFFu, need && alpha != 1.f) && __all_sync(0xFFFFFFFFu, ok)) {
       // rescale this warp's accumulator rows (PV_{j-1} has completed)
 #pragma unroll
       for (int cb = 0; cb < D; cb += 32) {
@@ -267,6 +282,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     __syncthreads();
     if (*abort_flag) break;
     // O += P V_j
+    last_o = j;
     if (tid == 0) {
       tc_fence_after();
       const uint32_t aV = smem_u32(smem + PrefillSmem::kV + st * 16384);
@@ -280,9 +296,15 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     }
   }
   cp_async_wait<0>();
-  if (n_tiles > 0 && !mbar_wait_bounded(bar_o, (uint32_t)((n_tiles - 1) & 1))) ok = false;
+  // drain: the phase of the last committed S and PV must have completed (a
+  // phase already seen completes the wait at once)
+  bool drained = true;
+  if (last_s >= 0 && !mbar_wait_bounded(bar_s, (uint32_t)(last_s & 1))) drained = false;
+  if (last_o >= 0 && !mbar_wait_bounded(bar_o, (uint32_t)(last_o & 1))) drained = false;
   tc_fence_after();
-  if (!ok || *abort_flag) {
+  const bool failed = __syncthreads_or(!ok || !drained || *abort_flag || last_o != n_tiles - 1);
+  const bool all_drained = !__syncthreads_or(!drained);
+  if (failed) {
     if (tid == 0) report_error(kErrTimeout);
   } else {
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -301,7 +323,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0 && all_drained) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace hga

@@ -336,15 +336,20 @@ hga_status hga_prefill_growing(const void* q, int32_t n_q_heads, int32_t n_queri
  *   == 0, else the phase-by-phase kernel), 1 = always the phase-by-phase kernel
  *   (the one hga_route and hga_attend use), 2 = the fused kernel where it
  *   applies. Both compute the same routed set and attention.
- *   HGA_OPT_PREFILL_KERNEL: which kernel runs the prefill attention. 0 =
- *   automatic (currently the one-tile kernel, the faster of the two on the
- *   2048-on-63488 workload), 1 = one 128-row query tile per CTA, 2 = two
- *   tiles per CTA sharing each gathered key tile (warp-specialised, Q and P in
- *   tensor memory) when the query heads per KV head are a multiple of 4, else
- *   one tile. Both compute the same attention.
+ *   HGA_OPT_TEST_EXPIRE_PREFILL_WAIT: a test hook for the failure path of the
+ *   prefill attention kernel. 0 = off (the default). v > 0 makes every CTA of
+ *   the next prefill attention launches treat its wait for key tile v - 1 (its
+ *   QK^T MMA) as expired AFTER that wait has really completed, so the kernel
+ *   takes its timeout exit with no MMA outstanding: it stops issuing, waits for
+ *   what it committed, releases tensor memory, writes no output row and
+ *   reports HGA_ERR_TIMEOUT (error bit 8) through hga_get_device_error.
+ *   Keep it 0 outside tests.
+ * The options are process-wide by design: they choose launch shapes for tuning
+ * and tests, not results (every choice computes the same routed set and
+ * attention, except the test hook, which only makes calls fail).
  * Returns HGA_ERR_INVALID_ARG for an unknown option or value.
  */
-enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2, HGA_OPT_PREFILL_KERNEL = 3 };
+enum { HGA_OPT_CTAS_PER_HEAD = 1, HGA_OPT_DECODE_KERNEL = 2, HGA_OPT_TEST_EXPIRE_PREFILL_WAIT = 4 };
 hga_status hga_set_launch_option(int32_t option, int32_t value);
 
 /*

@@ -120,6 +120,11 @@ def test_launch_option_validation():
         hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 17)
     with pytest.raises(hga.HgaError):
         hga.hga_set_launch_option(7, 1)
+    with pytest.raises(hga.HgaError):
+        hga.hga_set_launch_option(3, 1)  # no option 3: the prefill attention has one kernel
+    with pytest.raises(hga.HgaError):
+        hga.hga_set_launch_option(hga.HGA_OPT_TEST_EXPIRE_PREFILL_WAIT, -1)
+    hga.hga_set_launch_option(hga.HGA_OPT_TEST_EXPIRE_PREFILL_WAIT, 0)
     hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
 
 

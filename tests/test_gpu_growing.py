@@ -24,13 +24,6 @@ def hga():
     return m
 
 
-@pytest.fixture(params=[1, 2], ids=["one_tile_per_cta", "two_tiles_per_cta"])
-def pf_kernel(hga, request):
-    hga.hga_set_launch_option(hga.HGA_OPT_PREFILL_KERNEL, request.param)
-    yield request.param
-    hga.hga_set_launch_option(hga.HGA_OPT_PREFILL_KERNEL, 0)
-
-
 def dev_bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
 
@@ -90,7 +83,7 @@ def small(hq, hkv, L0, T, k=8, G=2):
                           n_new=T, block=64)
 
 
-def test_growing_prefill_small(hga, pf_kernel):
+def test_growing_prefill_small(hga):
     L0, T = 3000, 256
     w = small(32, 4, L0, T)
     pairs = [(b, h) for b in range(T // 64) for h in range(4)]
@@ -98,7 +91,7 @@ def test_growing_prefill_small(hga, pf_kernel):
     assert exact >= n - 1
 
 
-def test_growing_prefill_ragged_history(hga, pf_kernel):
+def test_growing_prefill_ragged_history(hga):
     # histories that are not multiples of 16 or of the chunk: segments of the
     # routed list straddle the cache / own-token boundary
     L0, T = 5077, 192

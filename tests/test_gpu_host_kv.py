@@ -1,15 +1,17 @@
 """Host-resident K/V (the pages' placement: the whole cache in host memory, only
 the routed rows moved to the GPU): the same kernels read K/V through the host
-link from pinned, mapped host memory, with the summaries in device memory. The
-results must equal those of the device-resident cache bit for bit (same
-kernels, same data), and the device-resident path is itself checked against
-the oracle in test_gpu_decode.py / test_gpu_paged.py."""
+link from pinned, mapped host memory, with the summaries in device memory.
+Checked against the CPU oracle (routed lists under the near-tie rule of
+tests/parity.py, attention over the list the GPU chose), and against the
+device-resident cache, which must give the same results bit for bit (same
+kernels, same data)."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
-from parity import bits
+from parity import assert_attention_close, assert_lse_close, bits, check_route
 
 pytestmark = pytest.mark.gpu
 
@@ -52,6 +54,24 @@ def test_host_resident_decode_equals_device_resident(hga):
     assert np.array_equal(bits(cs), bits(dev.chunk_sum)) and np.array_equal(bits(gs), bits(dev.group_sum))
     assert torch.equal(n_h, n_d) and torch.equal(idx_h, idx_d)
     assert torch.equal(out_h, out_d) and torch.equal(lse_h, lse_d)
+
+    # the host-resident results against the oracle, every (sequence, KV head)
+    idx_c, n_c = idx_h.cpu().numpy(), n_h.cpu().numpy()
+    out_c, lse_c = out_h.cpu().numpy(), lse_h.cpu().numpy()
+    R = 8
+    exact = 0
+    for b, L in enumerate(inp.seq_lens):
+        L = int(L)
+        for h in range(4):
+            K, V = np.ascontiguousarray(inp.k[b, h, :L]), np.ascontiguousarray(inp.v[b, h, :L])
+            qh = np.ascontiguousarray(inp.q[b, h * R:(h + 1) * R])
+            cs_o, gs_o = oracle.summaries(K, 128, 16)
+            toks = idx_c[b, h, :n_c[b, h]].astype(np.int64)
+            exact += check_route(toks, qh, cs_o, gs_o, L, 128, 16, 16, 4, f"host route b{b} h{h}")
+            ref, rl = oracle.attend(qh, K, V, toks, with_lse=True)
+            assert_attention_close(out_c[b, h * R:(h + 1) * R], ref, f"host decode b{b} h{h}")
+            assert_lse_close(lse_c[b, h * R:(h + 1) * R], rl, f"host decode lse b{b} h{h}")
+    assert exact >= 11
 
 
 def test_host_kv_pointer_rejects_unmapped_memory(hga):
