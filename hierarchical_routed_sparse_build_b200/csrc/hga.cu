@@ -13,6 +13,7 @@
 #include <cstring>
 
 #include "hga.h"
+#include "hga_balanced.cuh"
 #include "hga_common.cuh"
 #include "hga_decode.cuh"
 #include "hga_hisa.cuh"
@@ -25,7 +26,7 @@ namespace hga {
 namespace {
 
 std::atomic<int> g_ctas_per_head{0};
-std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 phase-by-phase, 2 fused
+std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 phase-by-phase, 2 fused, 3 route + balanced attention
 std::atomic<int> g_fail_at_tile{-1};  // test hook of the prefill attention kernel (-1: off)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -230,6 +231,137 @@ hga_status run_decode(RoutedArgs a, int D, int units, cudaStream_t stream) {
   if (DecodeSmem(D, a.n_pad, a.kcap, a.C / a.g).total > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
   const int P = pick_cluster(units);
   cudaError_t e = D == 128 ? launch_decode<128>(a, units, P, stream) : launch_decode<64>(a, units, P, stream);
+  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- balanced decode
+
+// Most tiles one unit can have at any length up to max_len (UnitTiles over L).
+int max_unit_tiles(const hga_kv* kv, const hga_params* p) {
+  int best = 0;
+  const int C = p->chunk;
+  // the count depends on L only through nf (capped at top_chunks + 2) and the tail
+  for (int L = kv->max_len; L >= 0 && L > kv->max_len - 2 * C; --L) {
+    const int t = UnitTiles(L, C, p->group, p->top_chunks, p->top_groups).total();
+    if (t > best) best = t;
+  }
+  const int small = UnitTiles(3 * C - 1 < kv->max_len ? 3 * C - 1 : kv->max_len, C, p->group, p->top_chunks,
+                              p->top_groups).total();
+  return best > small ? best : small;
+}
+
+// Routed tiles of one unit at most (the route kernel's list length).
+int max_routed_tiles(const hga_kv* kv, const hga_params* p) {
+  const int nf_max = kv->max_len / p->chunk;
+  const int cand = nf_max > 2 ? nf_max - 2 : 0;
+  const int r = cand < p->top_chunks ? cand : p->top_chunks;
+  return r * p->top_groups * (p->group / 16);
+}
+
+bool split_applies(const hga_kv* kv, const hga_params* p) {
+  return p->group % 16 == 0 && kv->batch <= kSplitMaxBatch;
+}
+
+// Workspace of the balanced decode, 256-byte aligned parts: tile lists, partial
+// states (one slot per CTA + unit), merge counts.
+struct SplitLayout {
+  size_t tiles, part, count, total;
+  int tile_stride, grid_max;
+  SplitLayout(const hga_kv* kv, const hga_params* p, int sms) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t units = (size_t)kv->batch * kv->n_kv_heads;
+    tile_stride = max_routed_tiles(kv, p);
+    if (tile_stride < 1) tile_stride = 1;
+    grid_max = 2 * sms;
+    tiles = 0;
+    part = up(tiles + units * (size_t)tile_stride * 4);
+    count = up(part + ((size_t)grid_max + units) * kPartFloats * 4);
+    total = up(count + units * 4);
+  }
+};
+
+int split_grid(const hga_kv* kv, const hga_params* p, int sms) {
+  // at least ~8 tiles per CTA, so that small problems do not spread over more
+  // CTAs (and partial merges) than they have work for
+  const int64_t t_max = (int64_t)kv->batch * kv->n_kv_heads * max_unit_tiles(kv, p);
+  int64_t gsz = t_max / 8;
+  if (gsz > 2 * sms) gsz = 2 * sms;
+  return gsz < 1 ? 1 : (int)gsz;
+}
+
+template <int D>
+cudaError_t launch_split(const RoutedArgs& a, const SplitArgs& sp, int units, int P, cudaStream_t stream) {
+  const RouteTilesSmem lay1(D, a.n_pad, a.kcap, a.C / a.g);
+  const BalancedSmem lay2(D, a.kv.batch, sp.grid);
+  auto k1 = route_tiles_kernel<D>;
+  auto k2 = balanced_attend_kernel<D>;
+  static std::atomic<int> smem1[kMaxDevices], smem2[kMaxDevices];
+  static std::atomic<bool> np_set[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (lay1.total > smem1[dev].load()) {
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, lay1.total)) != cudaSuccess)
+      return e;
+    smem1[dev].store(lay1.total);
+  }
+  if (lay2.total > smem2[dev].load()) {
+    if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, lay2.total)) != cudaSuccess)
+      return e;
+    smem2[dev].store(lay2.total);
+  }
+  if (P > 8 && !np_set[dev].load()) {
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess) return e;
+    np_set[dev].store(true);
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3((unsigned)(units * P), 1, 1);
+  cfg.blockDim = dim3(kRoutedThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)lay1.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&cfg, k1, a, sp)) != cudaSuccess) return e;
+  // the attention kernel is a programmatic dependent of the route kernel: it may
+  // start in free SM slots and attend sink / local tiles before the routes exist
+  cudaLaunchConfig_t cfg2;
+  std::memset(&cfg2, 0, sizeof cfg2);
+  cfg2.gridDim = dim3((unsigned)sp.grid, 1, 1);
+  cfg2.blockDim = dim3(kRoutedThreads, 1, 1);
+  cfg2.dynamicSmemBytes = (size_t)lay2.total;
+  cfg2.stream = stream;
+  cudaLaunchAttribute attr2[1];
+  attr2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr2[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg2.attrs = attr2;
+  cfg2.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg2, k2, a, sp);
+}
+
+hga_status run_split(const RoutedArgs& a, const hga_kv* kv, const hga_params* p, void* workspace, int D,
+                     cudaStream_t stream) {
+  if (RouteTilesSmem(D, a.n_pad, a.kcap, a.C / a.g).total > kMaxSmemPerCta ||
+      BalancedSmem(D, kv->batch, 2 * sm_count()).total > kMaxSmemPerCta)
+    return HGA_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  const SplitLayout lay(kv, p, sms);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  SplitArgs sp;
+  sp.tiles = reinterpret_cast<uint32_t*>(ws + lay.tiles);
+  sp.tile_stride = lay.tile_stride;
+  sp.part = reinterpret_cast<float*>(ws + lay.part);
+  sp.count = reinterpret_cast<int*>(ws + lay.count);
+  sp.grid = split_grid(kv, p, sms);
+  const int units = kv->batch * kv->n_kv_heads;
+  const int P = pick_cluster(units);
+  cudaError_t e = D == 128 ? launch_split<128>(a, sp, units, P, stream) : launch_split<64>(a, sp, units, P, stream);
   return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
 }
 
@@ -577,18 +709,9 @@ hga_status hga_attend(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
   return run_routed<kModeAttend>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
 }
 
-hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
-                      const void* group_sum, const hga_params* p, float* out, float* lse,
-                      int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream) {
-  hga_status s = check_kv(kv, true);
-  if (s != HGA_OK) return s;
-  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
-  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
-  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || group_sum == nullptr ||
-      !aligned16(chunk_sum) || !aligned16(group_sum) || out == nullptr)
-    return HGA_ERR_INVALID_ARG;
-  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
-  if (idx != nullptr && idx_stride < max_routed(kv, p)) return HGA_ERR_INVALID_ARG;
+static hga_status decode_impl(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                       const void* group_sum, const hga_params* p, float* out, float* lse, int32_t* idx,
+                       int32_t idx_stride, int32_t* n_idx, void* workspace, cudaStream_t stream) {
   RoutedArgs a;
   std::memset(&a, 0, sizeof a);
   a.kv = make_kv_view(kv);
@@ -603,9 +726,56 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
   a.idx_out = idx;
   a.n_idx_out = n_idx;
   a.idx_stride = idx ? idx_stride : 0;
-  if (g_decode_kernel.load() != 1 && p->group % 16 == 0)
+  // The route + balanced attention pair is opt-in: on B200 the fused kernel is
+  // faster at every batch measured (1, 4, 16 and 64 sequences of 64K tokens).
+  const int choice = g_decode_kernel.load();
+  if (workspace != nullptr && choice == 3 && split_applies(kv, p))
+    return run_split(a, kv, p, workspace, kv->head_dim, stream);
+  if (choice != 1 && p->group % 16 == 0)
     return run_decode(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
   return run_routed<kModeDecode>(a, kv->head_dim, kv->batch * kv->n_kv_heads, stream);
+}
+
+static hga_status check_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                        const void* group_sum, const hga_params* p, float* out, int32_t* idx, int32_t idx_stride,
+                        int32_t* n_idx) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || group_sum == nullptr ||
+      !aligned16(chunk_sum) || !aligned16(group_sum) || out == nullptr)
+    return HGA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
+  if (idx != nullptr && idx_stride < max_routed(kv, p)) return HGA_ERR_INVALID_ARG;
+  return HGA_OK;
+}
+
+hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                      const void* group_sum, const hga_params* p, float* out, float* lse,
+                      int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream) {
+  hga_status s = check_decode(q, n_q_heads, kv, chunk_sum, group_sum, p, out, idx, idx_stride, n_idx);
+  if (s != HGA_OK) return s;
+  return decode_impl(q, n_q_heads, kv, chunk_sum, group_sum, p, out, lse, idx, idx_stride, n_idx, nullptr, stream);
+}
+
+size_t hga_decode_workspace_size(const hga_kv* kv, int32_t n_q_heads, const hga_params* p) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK || check_heads(n_q_heads, kv) != HGA_OK)
+    return 0;
+  if (!split_applies(kv, p)) return 256;
+  return SplitLayout(kv, p, sm_count()).total;
+}
+
+hga_status hga_decode_ws(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                         const void* group_sum, const hga_params* p, float* out, float* lse, int32_t* idx,
+                         int32_t idx_stride, int32_t* n_idx, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+  hga_status s = check_decode(q, n_q_heads, kv, chunk_sum, group_sum, p, out, idx, idx_stride, n_idx);
+  if (s != HGA_OK) return s;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return HGA_ERR_INVALID_ARG;
+  if (workspace_bytes < hga_decode_workspace_size(kv, n_q_heads, p)) return HGA_ERR_INVALID_ARG;
+  return decode_impl(q, n_q_heads, kv, chunk_sum, group_sum, p, out, lse, idx, idx_stride, n_idx, workspace,
+                     stream);
 }
 
 int32_t hga_max_hisa_tokens(const hga_kv* kv, const hga_params* p, int32_t top_tokens) {
@@ -801,7 +971,7 @@ hga_status hga_set_launch_option(int32_t option, int32_t value) {
     return HGA_OK;
   }
   if (option == HGA_OPT_DECODE_KERNEL) {
-    if (value < 0 || value > 2) return HGA_ERR_INVALID_ARG;
+    if (value < 0 || value > 3) return HGA_ERR_INVALID_ARG;
     g_decode_kernel.store(value);
     return HGA_OK;
   }

@@ -57,7 +57,7 @@ struct DecodeSmem {
     cta_m = o;   o = up16(o + 4 * kGatherSlots);
     cta_l = o;   o = up16(o + 4 * kGatherSlots);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
-    hist = o;    o = up16(o + 4 * kBuckets);
+    hist = o;    o = up16(o + 4 * kHistWords);
     misc = o;    o = up16(o + 4 * 32);
     gstage = o;  o = up16(o + kRoutedWarps * gpc * D * 2);
     uni = o;

@@ -62,7 +62,7 @@ struct HisaSmem {
     cta_m = o;   o = up16(o + 4 * kGatherSlots);
     cta_l = o;   o = up16(o + 4 * kGatherSlots);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
-    hist = o;    o = up16(o + 4 * kBuckets);
+    hist = o;    o = up16(o + 4 * kHistWords);
     misc = o;    o = up16(o + 4 * 32);
     kred = o;    o = up16(o + 8 * (2 * kRoutedWarps + 2));
     tmm = o;     o = up16(o + 4 * (kTmmWarp + 2 * kRoutedWarps));
@@ -145,36 +145,6 @@ __device__ __forceinline__ float route_key_score(uint64_t key) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Warp 0 walks the histogram from the top bucket down and finds the bucket
-// holding the need-th key: misc[0] = that bucket, misc[1] = keys above it.
-template <int NB>
-__device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, int* misc) {
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x >= 32) return;
-  constexpr int PER = NB / 32;
-  int tot = 0;
-  for (int k = 0; k < PER; ++k) tot += hist[NB - 1 - PER * lane - k];
-  int incl = tot;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  const int excl = incl - tot;
-  if (excl < need && need <= incl) {
-    int acc = excl;
-    for (int k = 0; k < PER; ++k) {
-      const int bk = NB - 1 - PER * lane - k;
-      if (acc + hist[bk] >= need) {
-        misc[0] = bk;
-        misc[1] = acc;
-        break;
-      }
-      acc += hist[bk];
-    }
-  }
-}
-
 // Top r of n distinct route keys (1 <= r < n), written to sel[] as their ids in
 // the keys' storage order (the token keys are stored in ascending position, so
 // the kept positions come out ascending). lo and hi are the least and greatest
@@ -206,7 +176,7 @@ __device__ __forceinline__ void select_top_keys(const uint64_t* keys, int n, int
   int bstar = 0, members = 0;
   if (tid == 0) kred[2 * kRoutedWarps] = ~0ull;  // kth; ordered by the first barrier below
   for (;;) {
-    for (int i = tid; i < kTokBuckets; i += kRoutedThreads) hist[i] = 0;
+    for (int i = tid; i < hist_index(kTokBuckets); i += kRoutedThreads) hist[i] = 0;
     if (tid == 0) {
       misc[0] = 0;
       misc[1] = 0;
@@ -215,14 +185,14 @@ __device__ __forceinline__ void select_top_keys(const uint64_t* keys, int n, int
     __syncthreads();
     for (int i = tid; i < n; i += kRoutedThreads) {
       const int bk = member_bucket(keys[i]);
-      if (bk >= 0) atomicAdd(&hist[bk], 1);
+      if (bk >= 0) atomicAdd(&hist[hist_index(bk)], 1);
     }
     __syncthreads();
     find_boundary_bucket<kTokBuckets>(hist, need, misc);
     __syncthreads();
     bstar = misc[0];
     need -= misc[1];
-    members = hist[bstar];
+    members = hist[hist_index(bstar)];
     if (members <= kTokRankCap || level >= kTokRefine) break;
     // key range of the boundary bucket -> the next level's interval
     uint64_t mn = ~0ull, mx = 0ull;

@@ -47,7 +47,7 @@ struct BlockRouteSmem {
     keys = o;   o = up16(o + 8 * n_pad);
     sel = o;    o = up16(o + 4 * kcap);
     gmask = o;  o = up16(o + 4 * kcap);
-    hist = o;   o = up16(o + 4 * kBuckets);
+    hist = o;   o = up16(o + 4 * kHistWords);
     misc = o;   o = up16(o + 4 * 32);
     gsc = o;    o = up16(o + 4 * kcap * gpc);
     gstart = o; o = up16(o + 4 * kcap * gk);

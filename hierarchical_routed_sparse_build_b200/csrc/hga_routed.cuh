@@ -44,6 +44,11 @@ enum RoutedMode : int { kModeRoute = 1, kModeAttend = 2, kModeDecode = 3 };
 constexpr int kRoutedWarps = 6;
 constexpr int kRoutedThreads = kRoutedWarps * 32;
 constexpr int kBuckets = 1024;             // bucket-select histogram size
+// Histograms are stored with one padding word after every 32 buckets
+// (hist_index), so that warp lanes reading buckets a multiple of 32 apart hit
+// distinct shared-memory banks; kHistWords words hold kBuckets buckets.
+constexpr int kHistWords = kBuckets + kBuckets / 32;
+__host__ __device__ constexpr int hist_index(int b) { return b + (b >> 5); }
 // misc[] (32 ints): [0..5] select state, [8..15] per-warp min, [16..23] per-warp
 // max, [24..31] per-warp scan totals
 static_assert(kRoutedWarps <= 8, "misc[] holds at most 8 per-warp slots");
@@ -91,7 +96,7 @@ struct RoutedSmem {
     cta_m = o;   o = up16(o + 4 * kGatherSlots);
     cta_l = o;   o = up16(o + 4 * kGatherSlots);
     qfrag = o;   o = up16(o + 16 * 32 * (D / 32));
-    hist = o;    o = up16(o + 4 * kBuckets);
+    hist = o;    o = up16(o + 4 * kHistWords);
     misc = o;    o = up16(o + 4 * 32);
     // union: {keys, staging} during routing | per-warp tiles | partial outputs
     uni = o;
@@ -191,6 +196,46 @@ __device__ __forceinline__ void stream_rows(uint4* stage, int stage_rows, int n_
   cp_async_wait<0>();
 }
 
+// Warp 0 finds the bucket holding the need-th largest key (1 <= need <= keys
+// counted): misc[0] = that bucket, misc[1] = keys in the buckets above it. Lane l
+// sums the NB/32 buckets NB-1-(NB/32)l-k (k ascending = buckets descending), a
+// warp scan finds the lane whose range holds the need-th key, then one bucket
+// of that range per lane and a second scan find the bucket. The padded layout
+// makes both reads free of bank conflicts.
+template <int NB>
+__device__ __forceinline__ void find_boundary_bucket(const int* hist, int need, int* misc) {
+  static_assert(NB % 32 == 0 && NB / 32 <= 32, "one bucket range per lane, at most 32 buckets each");
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x & 31;
+  constexpr int PER = NB / 32;
+  int tot = 0;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) tot += hist[hist_index(NB - 1 - PER * lane - k)];
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int excl = incl - tot;
+  const uint32_t hit = __ballot_sync(0xFFFFFFFFu, excl < need && need <= incl);
+  const int L = __ffs(hit) - 1;
+  const int above = __shfl_sync(0xFFFFFFFFu, excl, L);
+  const int bk = NB - 1 - PER * L - lane;  // this lane's bucket of range L
+  const int v = lane < PER ? hist[hist_index(bk)] : 0;
+  int pre = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, pre, off);
+    if (lane >= off) pre += t;
+  }
+  const uint32_t hit2 = __ballot_sync(0xFFFFFFFFu, lane < PER && above + pre >= need);
+  if (lane == __ffs(hit2) - 1) {
+    misc[0] = bk;
+    misc[1] = above + pre - v;
+  }
+}
+
 // Top-r selection over n unique keys; keys[i] belongs to candidate chunk i+1
 // (key = order-preserving score bits << 32 | ~id, so larger key = higher score,
 // then lower id: the oracle's order). Finds the r-th largest key K_r exactly and
@@ -221,7 +266,7 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
     misc[8 + warp] = (int)lo;
     misc[16 + warp] = (int)hi;
   }
-  for (int i = tid; i < NB; i += kRoutedThreads) hist[i] = 0;
+  for (int i = tid; i < hist_index(NB); i += kRoutedThreads) hist[i] = 0;
   if (tid == 0) misc[2] = 0;
   __syncthreads();
   lo = 0xFFFFFFFFu;
@@ -233,35 +278,12 @@ __device__ __forceinline__ void select_top_chunks(const uint64_t* keys, int n, i
   }
   const float scale = (float)NB / ((float)(hi - lo) + 1.0f);
   auto bucket = [&](uint32_t u) { return min(NB - 1, (int)((float)(u - lo) * scale)); };
-  for (int i = tid; i < n; i += kRoutedThreads) atomicAdd(&hist[bucket((uint32_t)(keys[i] >> 32))], 1);
+  for (int i = tid; i < n; i += kRoutedThreads) atomicAdd(&hist[hist_index(bucket((uint32_t)(keys[i] >> 32)))], 1);
   __syncthreads();
-  if (warp == 0) {
-    constexpr int PER = NB / 32;
-    int tot = 0;
-    for (int k = 0; k < PER; ++k) tot += hist[NB - 1 - PER * lane - k];
-    int incl = tot;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    const int excl = incl - tot;
-    if (excl < r && r <= incl) {
-      int acc = excl;
-      for (int k = 0; k < PER; ++k) {
-        const int b = NB - 1 - PER * lane - k;
-        if (acc + hist[b] >= r) {
-          misc[0] = b;
-          misc[1] = acc;
-          break;
-        }
-        acc += hist[b];
-      }
-    }
-  }
+  find_boundary_bucket<NB>(hist, r, misc);
   __syncthreads();
   const int bstar = misc[0], need = r - misc[1];
-  const int members = hist[bstar];
+  const int members = hist[hist_index(bstar)];
   const bool in_scratch = members <= scratch_cap;
   if (in_scratch) {
     for (int i = tid; i < n; i += kRoutedThreads) {

@@ -9,8 +9,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (hga_append, hga_attend, hga_build_summaries, hga_decode, hga_decode_hisa, hga_max_hisa_tokens,
-               hga_max_routed_tokens, hga_route, hga_summary_bytes, make_kv, make_params)
+from . import (hga_append, hga_attend, hga_build_summaries, hga_decode_hisa, hga_decode_workspace_size, hga_decode_ws,
+               hga_max_hisa_tokens, hga_max_routed_tokens, hga_route, hga_summary_bytes, make_kv, make_params)
 
 
 def _dev_u16(a: np.ndarray, device) -> torch.Tensor:
@@ -60,6 +60,10 @@ class RoutedCache:
             self.group_sum = torch.zeros((batch, hkv, nc, gpc, d), dtype=torch.bfloat16, device=self.device)
         assert self.chunk_sum.numel() * 2 == cb and self.group_sum.numel() * 2 == gb
         self.idx_stride = hga_max_routed_tokens(self.kv, self.params)
+        # decode workspace (route lists and softmax partials of the balanced decode)
+        with torch.cuda.device(self.device):
+            self.ws_bytes = hga_decode_workspace_size(self.kv, n_q_heads, self.params)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
 
     # -- buffers -----------------------------------------------------------------
     def q_tensor(self, q) -> torch.Tensor:
@@ -121,6 +125,6 @@ class RoutedCache:
             out, lse = self.out_buffers()
         if want_idx and idx is None:
             idx, n_idx = self.idx_buffers()
-        hga_decode(q, self.n_q_heads, self.kv, self.chunk_sum, self.group_sum, self.params, out, lse,
-                   idx, self.idx_stride if idx is not None else 0, n_idx, stream)
+        hga_decode_ws(q, self.n_q_heads, self.kv, self.chunk_sum, self.group_sum, self.params, out, lse,
+                      idx, self.idx_stride if idx is not None else 0, n_idx, self.workspace, self.ws_bytes, stream)
         return (out, lse, idx, n_idx) if want_idx else (out, lse)

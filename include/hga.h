@@ -193,6 +193,34 @@ hga_status hga_decode(const void* q, int32_t n_q_heads, const hga_kv* kv, const 
                       int32_t* idx, int32_t idx_stride, int32_t* n_idx, cudaStream_t stream);
 
 /*
+ * Bytes of workspace hga_decode_ws needs for this cache and these parameters (0
+ * on invalid arguments). The size depends on the current device's SM count:
+ * query it with the device that will run the decode current.
+ */
+size_t hga_decode_workspace_size(const hga_kv* kv, int32_t n_q_heads, const hga_params* p);
+
+/*
+ * hga_decode with a caller-provided workspace (device memory, 256-byte aligned,
+ * at least hga_decode_workspace_size bytes; its contents on entry do not matter
+ * and on return are unspecified). Same arguments and results as hga_decode.
+ * With a workspace the decode can run as two kernels that balance the
+ * attention over the whole GPU (HGA_OPT_DECODE_KERNEL = 3): a route kernel
+ * (the chunk scores, chunk top-k and group top-G of hga_route, one
+ * thread-block cluster per (sequence, KV head)) writes the routed 16-token
+ * tiles of every (sequence, KV head) into the workspace, and an attention
+ * kernel cuts the tiles of all of them into equal slices, one per CTA,
+ * merging the softmax partials of a (sequence, KV head) that several CTAs
+ * share through the workspace. That pair applies when group % 16 == 0 and
+ * batch <= 4096. By default (option 0) the call runs hga_decode's kernel,
+ * which is faster on B200 at every batch measured, and leaves the workspace
+ * unused. Calls that share one workspace must not overlap on the GPU.
+ */
+hga_status hga_decode_ws(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                         const void* group_sum, const hga_params* p, float* out, float* lse, int32_t* idx,
+                         int32_t idx_stride, int32_t* n_idx, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
  * Chunked prefill. n_queries new tokens sit at positions cache_len ..
  * cache_len + n_queries - 1; their keys and values are already written into
  * the cache at those positions (kv->max_len >= cache_len + n_queries). The
@@ -331,11 +359,13 @@ hga_status hga_prefill_growing(const void* q, int32_t n_q_heads, int32_t n_queri
  *   HGA_OPT_CTAS_PER_HEAD: CTAs (one thread-block cluster) that cooperate on one
  *   (sequence, KV head) in hga_route / hga_attend / hga_decode; 0 = automatic,
  *   1..16 otherwise (above 8 needs non-portable cluster support).
- *   HGA_OPT_DECODE_KERNEL: which kernel runs hga_decode. 0 = automatic (the
- *   fused kernel that routes groups inside the attention warps when group % 16
- *   == 0, else the phase-by-phase kernel), 1 = always the phase-by-phase kernel
- *   (the one hga_route and hga_attend use), 2 = the fused kernel where it
- *   applies. Both compute the same routed set and attention.
+ *   HGA_OPT_DECODE_KERNEL: which kernels run hga_decode / hga_decode_ws. 0 =
+ *   automatic (the fused kernel that routes groups inside the attention warps
+ *   when group % 16 == 0, else the phase-by-phase kernel), 1 = always the
+ *   phase-by-phase kernel (the one hga_route and hga_attend use), 2 = the
+ *   fused kernel where it applies, 3 = the route + balanced attention pair
+ *   where it applies (hga_decode_ws only; elsewhere as 0). All compute the
+ *   same routed set and attention.
  *   HGA_OPT_TEST_EXPIRE_PREFILL_WAIT: a test hook for the failure path of the
  *   prefill attention kernel. 0 = off (the default). v > 0 makes every CTA of
  *   the next prefill attention launches treat its wait for key tile v - 1 (its

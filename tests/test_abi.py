@@ -223,3 +223,25 @@ def test_hisa_kept_list_is_bounded_by_the_candidates():
     kv, p = kv_desc(), params()
     assert hga._lib.hga_max_hisa_tokens(ctypes.byref(kv), ctypes.byref(p), 10_000_000) == \
         max(oracle.hisa_candidates(L, 128, 32) for L in range(65536 - 256, 65537))
+
+
+def raw_decode_ws(kv, p, ws=FAKE, nbytes=1 << 30, hq=32):
+    return hga._lib.hga_decode_ws(FAKE, hq, ctypes.byref(kv), FAKE, FAKE, ctypes.byref(p), FAKE, None, None, 0,
+                                  None, ws, nbytes, None)
+
+
+def test_decode_workspace_size_and_validation():
+    kv, p = kv_desc(batch=64), params()
+    n = hga.hga_decode_workspace_size(kv, 32, p)
+    units, sms = 64 * 4, 148  # no device here: the library assumes a B200's 148 SMs
+    # routed tile lists (32 chunks x 4 groups x one 16-token tile each), one partial
+    # softmax state per (CTA of a 2-per-SM grid + unit), one merge count per unit
+    floor = units * 32 * 4 * 4 + (2 * sms + units) * 8 * 130 * 4 + units * 4
+    assert floor <= n <= floor + 3 * 256
+    # groups that are not whole 16-token tiles run the one-kernel decode: no real workspace
+    assert hga.hga_decode_workspace_size(kv, 32, params(group=8)) == 256
+    assert hga._lib.hga_decode_workspace_size(ctypes.byref(kv_desc(head_dim=96)), 32, ctypes.byref(p)) == 0
+    assert raw_decode_ws(kv, p, ws=0) == INVALID                     # no workspace
+    assert raw_decode_ws(kv, p, ws=FAKE + 16) == INVALID             # not 256-byte aligned
+    assert raw_decode_ws(kv, p, nbytes=n - 1) == INVALID             # too small
+    assert raw_decode_ws(kv_desc(head_dim=96), p) == UNSUPPORTED     # the decode's own checks still apply

@@ -23,6 +23,15 @@ def hga():
     return m
 
 
+@pytest.fixture(params=[2, 3], ids=["fused", "balanced"])
+def decode_path(hga, request):
+    """Run a test with the fused one-kernel decode and with the route + balanced
+    attention pair (RoutedCache.decode calls hga_decode_ws)."""
+    hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, request.param)
+    yield request.param
+    hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, 0)
+
+
 def cache_for(hga, w, k, v, lens, page_table=None):
     from hierarchical_routed_sparse_build_b200.runtime import RoutedCache
     c = RoutedCache(k, v, lens, chunk=w.chunk, group=w.group, top_chunks=w.top_chunks,
@@ -104,33 +113,33 @@ def run_and_check(hga, w, inp, units=None, check_summaries=True):
     return exact, len(refs)
 
 
-def test_tiny_decode_4k(hga):
+def test_tiny_decode_4k(hga, decode_path):
     w = synth.TINY_DECODE_4K
     inp = synth.decode_inputs(w)
     exact, n = run_and_check(hga, w, inp)
     assert exact == n
 
 
-def test_decode_16k(hga):
+def test_decode_16k(hga, decode_path):
     w = synth.DECODE_16K
     exact, n = run_and_check(hga, w, synth.decode_inputs(w))
     assert exact >= n - 1
 
 
-def test_decode_64k(hga):
+def test_decode_64k(hga, decode_path):
     w = synth.DECODE_64K
     exact, n = run_and_check(hga, w, synth.decode_inputs(w))
     assert exact >= n - 1
 
 
 @pytest.mark.parametrize("L", [4096, 8192, 32768])
-def test_decode_sweep_lengths(hga, L):
+def test_decode_sweep_lengths(hga, decode_path, L):
     w = synth.with_len(synth.DECODE_64K, L)
     exact, n = run_and_check(hga, w, synth.decode_inputs(w))
     assert exact >= n - 1
 
 
-def test_ragged_batch_edge_lengths(hga):
+def test_ragged_batch_edge_lengths(hga, decode_path):
     # dense cases (fewer than 3 full chunks), exact chunk multiples, ragged tails,
     # a single token, and an empty sequence, in one batch
     w = synth.Workload("edge", 1, 32, 4, 128, 0, 128, 16, 4, 2, -1, 7)
@@ -143,13 +152,13 @@ def test_ragged_batch_edge_lengths(hga):
 
 
 @pytest.mark.parametrize("hq,hkv,d", [(4, 4, 128), (12, 4, 64), (6, 2, 128), (8, 1, 64)])
-def test_head_shapes(hga, hq, hkv, d):
+def test_head_shapes(hga, decode_path, hq, hkv, d):
     w = synth.Workload(f"heads{hq}x{hkv}x{d}", 1, hq, hkv, d, 3000, 64, 16, 6, 2, -1, 11)
     inp = synth.decode_inputs(w, lengths=[3000, 2500], max_len=3000)
     run_and_check(hga, w, inp)
 
 
-def test_full_coverage_is_dense_attention(hga):
+def test_full_coverage_is_dense_attention(hga, decode_path):
     # top_chunks >= candidates and top_groups = C/g: every token is routed, so the
     # output must be dense attention over the whole context.
     w = synth.Workload("full", 1, 32, 4, 128, 2000, 64, 16, 1000, 4, -1, 13)
@@ -165,7 +174,7 @@ def test_full_coverage_is_dense_attention(hga):
             assert_attention_close(out[b, h * 8:(h + 1) * 8].cpu().numpy(), ref, f"dense b{b} h{h}")
 
 
-@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("kernel", [1, 2, 3])
 @pytest.mark.parametrize("ctas", [1, 2, 3, 8, 16])
 def test_cluster_sizes_agree(hga, ctas, kernel):
     w = synth.with_len(synth.DECODE_64K, 16384)
@@ -211,7 +220,7 @@ def test_one_cta_per_head_ragged_and_paged(hga):
 
 
 @pytest.mark.parametrize("group,chunk,top_groups", [(8, 128, 4), (32, 128, 2), (16, 64, 4), (16, 256, 3)])
-def test_group_sizes(hga, group, chunk, top_groups):
+def test_group_sizes(hga, decode_path, group, chunk, top_groups):
     # g = 8 runs the phase-by-phase kernel (a 16-token tile spans two groups);
     # g = 32 and chunk 256 run the fused kernel with two tiles per group and 16
     # groups per chunk; top_groups = C/g (all groups) runs its whole-chunk path
@@ -246,7 +255,7 @@ def test_attend_arbitrary_token_order_and_ragged_list(hga):
         assert_lse_close(lse[0, h * 8:(h + 1) * 8].cpu().numpy(), rl, f"lse h{h}")
 
 
-def test_device_errors_are_reported_not_faulted(hga):
+def test_device_errors_are_reported_not_faulted(hga, decode_path):
     w = synth.Workload("err", 1, 8, 1, 128, 1024, 128, 16, 2, 2, -1, 19)
     inp = synth.decode_inputs(w, lengths=[1024, 512])
     c = cache_for(hga, w, inp.k, inp.v, inp.seq_lens)

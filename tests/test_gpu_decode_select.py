@@ -6,11 +6,12 @@ vector, so every chunk score and every group score is bit-identical on the GPU
 (the same dot products in the same order for every row) and in the oracle. The
 tie rule (higher score first, then lower chunk / group index) then fixes the
 routed list exactly: chunks 1..k, groups 0..G-1. With 638 candidate chunks all
-in one histogram bucket, the fused decode's select cannot rank the boundary
-bucket in its 512-key shared-memory area and takes its fallback scan over all
-keys; the phase-by-phase kernel (hga_route) ranks them in its larger area.
-Both must give the oracle's list bit for bit, at one and at eight CTAs per
-(sequence, KV head).
+in one histogram bucket, the select of the fused decode and of the balanced
+pair's route kernel cannot rank the boundary bucket in its 512-key
+shared-memory area and takes its fallback scan over all keys; the
+phase-by-phase kernel (hga_route) ranks them in its larger area. All must give
+the oracle's list bit for bit, at one and at eight CTAs per (sequence, KV
+head).
 
 Benchmark configuration: 64K-token sequences decoded with one CTA per
 (sequence, KV head), the shape the automatic choice takes for a batch of 64;
@@ -80,7 +81,7 @@ def tied_cache(hga):
     return dict(c=c, q=c.q_tensor(q), lens=lens, want=want, R=R)
 
 
-@pytest.mark.parametrize("kernel", [1, 2], ids=["phase_by_phase", "fused"])
+@pytest.mark.parametrize("kernel", [1, 2, 3], ids=["phase_by_phase", "fused", "balanced"])
 @pytest.mark.parametrize("ctas", [1, 8])
 def test_all_tied_scores_keep_the_lowest_ids(hga, tied_cache, ctas, kernel):
     c, q, R = tied_cache["c"], tied_cache["q"], tied_cache["R"]
@@ -103,9 +104,11 @@ def test_all_tied_scores_keep_the_lowest_ids(hga, tied_cache, ctas, kernel):
         assert_lse_close(lse[b, sl], rl, f"tied decode lse b{b} h{h}")
 
 
-def test_decode_64k_at_the_benchmark_launch_shape(hga):
+@pytest.mark.parametrize("kernel", [2, 3], ids=["fused", "balanced"])
+def test_decode_64k_at_the_benchmark_launch_shape(hga, kernel):
     """16 sequences of 65536 tokens (8 drawn, each repeated in separate memory, as
-    the benchmark builds its batch), one CTA per (sequence, KV head)."""
+    the benchmark builds its batch), one CTA per (sequence, KV head) in the fused
+    kernel (and in the route kernel of the balanced pair)."""
     from hierarchical_routed_sparse_build_b200.runtime import RoutedCache
     w = synth.DECODE_64K
     B = 16
@@ -115,11 +118,13 @@ def test_decode_64k_at_the_benchmark_launch_shape(hga):
     c.build_summaries()
     q = c.q_tensor(inp.q)
     hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 1)
+    hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, kernel)
     try:
         out, lse, idx, n_idx = c.decode(q, want_idx=True)
         no_device_error(hga)
     finally:
         hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
+        hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, 0)
     idx, n_idx, out, lse = idx.cpu().numpy(), n_idx.cpu().numpy(), out.cpu().numpy(), lse.cpu().numpy()
     R = w.n_q_heads // w.n_kv_heads
     L = w.ctx_len
@@ -142,5 +147,9 @@ def test_decode_64k_at_the_benchmark_launch_shape(hga):
             assert_attention_close(out[b, sl], ref, f"decode b{b} h{h}")
             assert_lse_close(lse[b, sl], rl, f"decode lse b{b} h{h}")
     assert exact >= total - 2
-    # the repeated sequences (same values, other memory) must give the same bits
-    assert np.array_equal(out[:8], out[8:]) and np.array_equal(lse[:8], lse[8:])
+    # the repeated sequences (same values, other memory) route identically; the
+    # fused kernel then gives the same bits (the balanced pair cuts their tiles
+    # into other slices, so its merges may round differently)
+    assert np.array_equal(idx[:8], idx[8:])
+    if kernel == 2:
+        assert np.array_equal(out[:8], out[8:]) and np.array_equal(lse[:8], lse[8:])

@@ -38,10 +38,15 @@ def test_paged_lengths_and_table(setup):
     assert len(np.unique(used)) == used.size == inp.k_pool.shape[0]
 
 
-def test_paged_decode_matches_oracle(setup):
+@pytest.mark.parametrize("kernel", [2, 3], ids=["fused", "balanced"])
+def test_paged_decode_matches_oracle(setup, kernel):
     hga, w, inp, c = setup
     q = c.q_tensor(inp.q)
-    out, lse, idx, n_idx = c.decode(q, want_idx=True)
+    hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, kernel)
+    try:
+        out, lse, idx, n_idx = c.decode(q, want_idx=True)
+    finally:
+        hga.hga_set_launch_option(hga.HGA_OPT_DECODE_KERNEL, 0)
     st, b = hga.hga_get_device_error()
     assert st == 0, b
     cs_gpu, gs_gpu = bits(c.chunk_sum), bits(c.group_sum)

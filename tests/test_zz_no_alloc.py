@@ -107,11 +107,13 @@ def test_prefill_noalloc_at_its_limit():
     assert torch.equal(got, ref), "a problem that fills the array exactly differs from hga_prefill"
     # one block more is over the limit: refused before anything is enqueued
     T = 4160
+    k = torch.zeros((1, 8, 1663 + T, 128), dtype=torch.bfloat16, device="cuda")
+    kv = hga.make_kv(k, k, pr["lens"], n_kv_heads=8, head_dim=128, max_len=1663 + T, batch=1)
     q = torch.zeros((T, 16, 128), dtype=torch.bfloat16, device="cuda")
     out = torch.full((T, 16, 128), 3.0, dtype=torch.float32, device="cuda")
-    assert hga.hga_prefill_workspace_size(pr["kv"], 16, T, 64, 1663, pr["p"]) > 2 << 20
+    assert hga.hga_prefill_workspace_size(kv, 16, T, 64, 1663, pr["p"]) == (2 << 20) + 8 * 1024 * 4
     with pytest.raises(hga.HgaError) as e:
-        hga.hga_prefill_noalloc(q, 16, T, 64, pr["kv"], 1663, pr["cs"], pr["gs"], pr["p"], out)
+        hga.hga_prefill_noalloc(q, 16, T, 64, kv, 1663, pr["cs"], pr["gs"], pr["p"], out)
     assert e.value.status == 2  # HGA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert torch.all(out == 3.0)
