@@ -24,6 +24,7 @@ import subprocess
 import sys
 import threading
 import time
+import types
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -97,20 +98,17 @@ def kernel_source_hash(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(profile="decode_64k_decode_kernel.md", names=DECODE_SOURCES):
-    """DRAM bytes per launch from a committed ncu summary, if it covers the current sources."""
-    import re
-
-    path = os.path.join(ROOT, "profiles", profile)
+def profiled_traffic(profile="decode_64k_decode_kernel", names=DECODE_SOURCES):
+    """DRAM bytes per launch from a committed ncu record (profiles/<profile>.json), if it was taken on the
+    current sources (its source_hash equals kernel_source_hash(names)); None otherwise."""
     try:
-        text = open(path).read()
-    except OSError:
+        with open(os.path.join(ROOT, "profiles", profile + ".json")) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(names):
+    if rec.get("source_hash") != kernel_source_hash(names):
         return None
-    return int(m_bytes.group(1))
+    return int(rec["traffic_bytes_per_launch"])
 
 
 def bf16_peak():
@@ -131,7 +129,7 @@ def prefill_flops(routed_total: int, n_pairs: int, w=synth.PREFILL_64K) -> int:
     return 4 * w.head_dim * R * keys
 
 
-def run_prefill(dev, steps: int, warmup: int):
+def run_prefill(dev, steps: int, warmup: int, cpu_seconds: float | None = None):
     """Time hga_prefill on the 2048-new-token, 63488-token-cache workload."""
     import torch
 
@@ -209,7 +207,8 @@ def run_prefill(dev, steps: int, warmup: int):
                      "achieved": round(attn_tf, 1), "peak": burst, "peak_kind": f"{kind} bf16 burst",
                      "unit": "TFLOP/s", "frac": round(attn_tf / burst, 4),
                      "frac_of_sustained": round(attn_tf / sustained, 4),
-                     "traffic": profiled_traffic("prefill_64k_attn_kernel.md", PREFILL_SOURCES)},
+                     "traffic": profiled_traffic("prefill_64k_attn_kernel", PREFILL_SOURCES)},
+        **({"cpu_baseline": oracle_prefill_baseline(inp, w, cpu_seconds)} if cpu_seconds else {}),
         "growing_history": {"what": "hga_prefill_growing: block b routes over its whole history "
                                     "[0, 63488 + 64 b), earlier blocks of the call included",
                             "ms_per_step": round(grow, 4), "tokens_per_s": round(T / (grow * 1e-3), 1),
@@ -336,6 +335,73 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
+def oracle_rate(items, fn, seconds: float, threads: int | None = None):
+    """Run fn over items (repeating the list) on host threads for about `seconds`;
+    returns (items done per second, threads, items done, elapsed seconds)."""
+    threads = threads or os.cpu_count() or 1
+    done = 0
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        while True:
+            list(ex.map(fn, items))
+            done += len(items)
+            if time.perf_counter() - t0 >= seconds:
+                break
+    dt = time.perf_counter() - t0
+    return done / dt, threads, done, dt
+
+
+def oracle_decode_baseline(inp, w, seconds: float, contiguous=None) -> dict:
+    """The oracle's decode (routing on prebuilt summaries, then attention) for every (sequence, KV head)
+    of a decode input, on all host threads; queries/s (one query = all KV heads of one sequence)."""
+    import oracle
+
+    R = w.n_q_heads // w.n_kv_heads
+    B = len(inp.seq_lens)
+    prep = {}
+    for b in range(B):
+        L = int(inp.seq_lens[b])
+        K, V = contiguous(b) if contiguous else (inp.k[b, :, :L], inp.v[b, :, :L])
+        for h in range(w.n_kv_heads):
+            Kh, Vh = np.ascontiguousarray(K[h]), np.ascontiguousarray(V[h])
+            prep[(b, h)] = (Kh, Vh, oracle.summaries(Kh, w.chunk, w.group), L)
+
+    def one(u):
+        b, h = u
+        Kh, Vh, (cs, gs), L = prep[u]
+        qh = inp.q[b, h * R:(h + 1) * R]
+        tok = oracle.route(qh, cs, gs, L, w.chunk, w.group, w.top_chunks, w.top_groups)
+        oracle.attend(qh, Kh, Vh, tok)
+
+    rate, threads, done, dt = oracle_rate(list(prep), one, seconds)
+    return {"value": round(rate / w.n_kv_heads, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} (sequence, KV head) decodes of this input ({done / w.n_kv_heads:.0f} queries) in "
+                      f"{dt:.1f} s, summaries prebuilt"}
+
+
+def oracle_prefill_baseline(inp, w, seconds: float, pairs=((0, 0), (13, 1), (31, 3), (20, 2))) -> dict:
+    """The oracle's prefill (block-max routing, then attention over the routed cache set plus the block's
+    causal prefix) on a few (block, KV head) pairs of the same input; new tokens/s."""
+    import oracle
+
+    R = w.n_q_heads // w.n_kv_heads
+    L0 = inp.cache_len
+    sums = {h: oracle.summaries(np.ascontiguousarray(inp.k[0, h, :L0]), w.chunk, w.group) for h in range(w.n_kv_heads)}
+
+    def one(pair):
+        blk, h = pair
+        qb = np.ascontiguousarray(inp.q[blk * w.block:(blk + 1) * w.block, h * R:(h + 1) * R])
+        cs, gs = sums[h]
+        tok = oracle.route(qb, cs, gs, L0, w.chunk, w.group, w.top_chunks, w.top_groups)
+        oracle.prefill_block(qb, inp.k[0, h], inp.v[0, h], tok, P=L0 + w.block * blk)
+
+    rate, threads, done, dt = oracle_rate(list(pairs), one, seconds)
+    return {"value": round(rate * w.block / w.n_kv_heads, 1), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} (block of {w.block} queries, KV head) pairs of the 2048-on-63488 prefill in {dt:.1f} s "
+                      "(summaries prebuilt); tokens/s = pairs/s x 64 / 4 KV heads"}
+
+
 def cpu_baseline_record(inp, w, seconds: float, single_seconds: float = 3.0) -> dict:
     """The oracle on every host thread (the baseline value) and, on a short sample, on one thread."""
     v, cores, sample = oracle_queries_per_s(inp, w, seconds)
@@ -387,7 +453,7 @@ def run_summaries(hga, cache, timed, B: int, n: int = 5) -> dict:
         return {"error": f"{type(exc).__name__}: {exc}"}
 
 
-def run_paged_batch(hga, RoutedCache, dev, timed, n: int) -> dict:
+def run_paged_batch(hga, RoutedCache, dev, timed, n: int, cpu_seconds: float | None = None) -> dict:
     """The batched decode on a paged pool: 16 ragged sequences of 4K-64K tokens (seeded lengths), page =
     chunk = 128 tokens, shuffled page table, L2 flushed between steps. A failure here is recorded in the
     object rather than ending the run."""
@@ -415,7 +481,41 @@ def run_paged_batch(hga, RoutedCache, dev, timed, n: int) -> dict:
                 "lengths": {"min": min(lens), "max": max(lens), "total": sum(lens)},
                 "us_per_step": round(step_ms * 1e3, 2), "queries_per_s": round(len(lens) / (step_ms * 1e-3)),
                 "alg_bytes_per_step": nbytes, "GB_s": round(nbytes / (step_ms * 1e-3) / 1e9, 1),
-                "frac_hbm": round(nbytes / (step_ms * 1e-3) / 1e9 / hbm, 4)}
+                "frac_hbm": round(nbytes / (step_ms * 1e-3) / 1e9 / hbm, 4),
+                **({"cpu_baseline": oracle_decode_baseline(pin, wp, cpu_seconds, contiguous=pin.contiguous)}
+                   if cpu_seconds else {})}
+    except Exception as exc:  # recorded, so that the rest of the line is still printed
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
+def run_config(hga, RoutedCache, dev, timed, w, n: int, cpu_seconds: float | None) -> dict:
+    """One decode configuration as its workload states it (batch 1), L2 flushed between steps, with the
+    oracle timed on the same input beside it. A failure is recorded in the object."""
+    try:
+        inp = synth.decode_inputs(w)
+        c = RoutedCache(inp.k, inp.v, inp.seq_lens, chunk=w.chunk, group=w.group, top_chunks=w.top_chunks,
+                        top_groups=w.top_groups, n_q_heads=w.n_q_heads, device=dev)
+        c.build_summaries()
+        q = c.q_tensor(inp.q)
+        out, lse = c.out_buffers()
+        for _ in range(3):
+            c.decode(q, out, lse)
+        ms = statistics.median(timed(n, lambda: c.decode(q, out, lse)))
+        st, bits = hga.hga_get_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error bits {bits}")
+        L = int(inp.seq_lens[0])
+        nbytes = decode_bytes(L, w)
+        hbm, _ = peaks()
+        res = {"what": f"{w.name}: batch {len(inp.seq_lens)}, {w.n_q_heads} q / {w.n_kv_heads} KV heads, d {w.head_dim}, "
+                       f"L {L}, chunk {w.chunk}, group {w.group}, top-{w.top_chunks} chunks + sink + local, "
+                       f"top-{w.top_groups} groups; one fused decode launch per query",
+               "us_per_query": round(ms * 1e3, 2), "queries_per_s": round(1.0 / (ms * 1e-3)),
+               "alg_bytes_per_query": nbytes, "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 2),
+               "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 5)}
+        if cpu_seconds:
+            res["cpu_baseline"] = oracle_decode_baseline(inp, w, cpu_seconds)
+        return res
     except Exception as exc:  # recorded, so that the rest of the line is still printed
         return {"error": f"{type(exc).__name__}: {exc}"}
 
@@ -483,22 +583,56 @@ def run_gpu(args, rank: int, world: int, dist):
     ms_per_step = total_ms / args.steps
     value = weak_scaling_rate(B, world, args.steps, total_ms)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: q copied in from pinned
+    # host memory and out/lse copied back every step, double-buffered on a copy
+    # stream so that step i+1's upload and step i's download run under decodes
     q_host = torch.from_numpy(inp.q.view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    q_dev = torch.empty_like(q)
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    lse_host = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    q_dev = [torch.empty_like(q) for _ in range(2)]
+    o_dev = [torch.empty_like(out) for _ in range(2)]
+    l_dev = [torch.empty_like(lse) for _ in range(2)]
+    copy = torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
+    up_done, dec_done, down_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step():
-        q_dev.copy_(q_host, non_blocking=True)
-        cache.decode(q_dev, out, lse)
-        out_host.copy_(out, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
+    def e2e_run(n):
+        """n end-to-end steps; returns their device time (ms) from the first upload to the last download."""
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.max()
+        t_start.record(stream)
+        copy.wait_event(t_start)
+        with torch.cuda.stream(copy):
+            q_dev[0].copy_(q_host, non_blocking=True)
+            up_done[0].record(copy)
+        for i in range(n):
+            sl = i % 2
+            if i + 1 < n:
+                with torch.cuda.stream(copy):
+                    if i >= 1:
+                        copy.wait_event(dec_done[1 - sl])  # decode i-1 has read that q buffer
+                    q_dev[1 - sl].copy_(q_host, non_blocking=True)
+                    up_done[1 - sl].record(copy)
+            stream.wait_event(up_done[sl])
+            if i >= 2:
+                stream.wait_event(down_done[sl])  # step i-2's outputs have left that buffer
+            cache.decode(q_dev[sl], o_dev[sl], l_dev[sl])
+            dec_done[sl].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(dec_done[sl])
+                out_host[sl].copy_(o_dev[sl], non_blocking=True)
+                lse_host[sl].copy_(l_dev[sl], non_blocking=True)
+                down_done[sl].record(copy)
+        stream.wait_stream(copy)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        return t_start.elapsed_time(t_end)
 
-    for _ in range(3):
-        e2e_step()
-    e2e_times = timed(args.steps, e2e_step)
-    e2e_ms = max_over_ranks(float(sum(e2e_times)), dist, dev)
+    e2e_run(3)
+    e2e_ms = max_over_ranks(e2e_run(args.steps), dist, dev)
+    got = out_host[(args.steps - 1) % 2]
+    if not torch.equal(got, out.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-timed decode of the same queries")
 
     # batch-1 latency and the context-length sweep (same kernels, same cache)
     sweep = {}
@@ -511,12 +645,17 @@ def run_gpu(args, rank: int, world: int, dist):
     cs1, gs1 = cache.chunk_sum[:1], cache.group_sum[:1]
     lat = timed(args.steps, lambda: hga_decode(q1, w.n_q_heads, kv1, cs1, gs1, cache.params, out1, lse1))
     hbm, peak_kind = peaks()
+    cpu_s = args.cpu_point_seconds if (not args.no_cpu_baseline and world == 1) else None
     for L in SWEEP:
         cache.seq_lens.fill_(L)
         tl = timed(max(10, args.steps // 4), step)
         ms = statistics.median(tl)
         sweep[str(L)] = {"queries_per_s": round(B / (ms / 1e3)), "GB_s": round(B * decode_bytes(L) / (ms / 1e3) / 1e9, 1),
                          "frac_hbm": round(B * decode_bytes(L) / (ms / 1e3) / 1e9 / hbm, 4)}
+        if cpu_s:
+            # the same queries on the first two distinct sequences cut to length L
+            sub = types.SimpleNamespace(q=inp.q[:2], k=inp.k[:2], v=inp.v[:2], seq_lens=np.full(2, L, np.int32))
+            sweep[str(L)]["cpu_baseline"] = oracle_decode_baseline(sub, w, cpu_s)
     cache.seq_lens.copy_(lens_saved)
     st, bits = hga.hga_get_device_error()
     if st != 0:
@@ -562,7 +701,7 @@ def run_gpu(args, rank: int, world: int, dist):
             "GB_s": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9, 1),
             "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4),
             "traffic": (lambda t: None if t is None else t * B // 64)(
-                profiled_traffic("hisa_64k_hisa_decode_kernel.md", HISA_SOURCES))}
+                profiled_traffic("hisa_64k_hisa_decode_kernel", HISA_SOURCES))}
 
     # host-resident K/V (the pages' placement): 8 of the sequences in pinned, mapped host
     # memory, summaries in HBM; the decode kernel reads only the routed rows over the host link
@@ -597,8 +736,10 @@ def run_gpu(args, rank: int, world: int, dist):
     achieved = alg / mean_launch_s / 1e9
     srt = sorted(times)
     pct = lambda p: srt[min(len(srt) - 1, int(round(p / 100 * (len(srt) - 1))))]
-    prefill = None if args.no_prefill else run_prefill(dev, max(5, args.steps // 10), args.warmup)
-    paged = run_paged_batch(hga, RoutedCache, dev, timed, max(10, args.steps // 2))
+    prefill = None if args.no_prefill else run_prefill(dev, max(5, args.steps // 10), args.warmup, cpu_s)
+    paged = run_paged_batch(hga, RoutedCache, dev, timed, max(10, args.steps // 2), cpu_s)
+    configs = {w_.name: run_config(hga, RoutedCache, dev, timed, w_, max(10, args.steps // 2), cpu_s)
+               for w_ in (synth.TINY_DECODE_4K, synth.DECODE_16K)}
     summaries = run_summaries(hga, cache, timed, B)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -619,7 +760,10 @@ def run_gpu(args, rank: int, world: int, dist):
                      "alg_bytes_per_query": decode_bytes(w.ctx_len), "alg_bytes_per_launch": alg},
         "e2e": {"value": round(weak_scaling_rate(B, world, args.steps, e2e_ms), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_host.numel() * 2),
-                "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4)},
+                "d2h_bytes_per_step": int(out_host[0].numel() * 4 + lse_host[0].numel() * 4),
+                "how": "RoutedCache.decode per step; q uploaded from pinned host memory and out/lse downloaded "
+                       "every step on a second stream, double-buffered (step i+1's upload and step i's download "
+                       "overlap decode i); timed from the first upload to the last download"},
         "clocks": clocks.summary(),
         "gpu_launches": args.steps,
         "latency_ms": {"p50": round(pct(50), 5), "p95": round(pct(95), 5), "p99": round(pct(99), 5)},
@@ -629,6 +773,7 @@ def run_gpu(args, rank: int, world: int, dist):
         "host_resident_kv": host_kv,
         "block_then_token": hisa,
         "paged_batch": paged,
+        "configs": configs,
         "summaries": summaries,
         "prefill": prefill,
     }
@@ -645,6 +790,8 @@ def main():
     ap.add_argument("--ctas", type=int, default=0, help="CTAs per (sequence, KV head); 0 = automatic")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-point-seconds", type=float, default=2.0,
+                    help="oracle seconds beside each configuration, sweep point, the paged batch and prefill")
     ap.add_argument("--traffic", type=float, default=None, help="ncu dram bytes per launch, if measured")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement")
