@@ -70,10 +70,12 @@ HISA_SOURCES = DECODE_SOURCES + ("hga_hisa.cuh",)
 HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (below the 2304 the two-level route keeps)
 
 
-def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64) -> int:
+def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64, reread: bool = False) -> int:
     """Algorithmic HBM bytes of one block-then-token decode query (all KV heads): candidate chunk
-    summaries, K of every candidate token (the token step scores them), K and V of the kept tokens,
-    q, out and lse."""
+    summaries, K of every candidate token (the token step scores them; that covers the kept tokens' K),
+    V of the kept tokens (K and V when every candidate is kept, the token step then being skipped), q,
+    out and lse. reread=True adds what the kernel reads beyond that: the kept tokens' K a second time
+    in its attention phase (the token step keeps only head-summed scores)."""
     C, d, hkv, hq = w.chunk, w.head_dim, w.n_kv_heads, w.n_q_heads
     nf = L // C
     if nf <= 2:
@@ -83,7 +85,8 @@ def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64) -> int:
         n_ct = C + min(w.top_chunks, cand) * C + (L - (nf - 1) * C)
     kept = min(k_tok, n_ct)
     scored_k = n_ct if n_ct > k_tok else 0
-    return (cand * hkv * d * 2 + scored_k * hkv * d * 2 + kept * hkv * d * 2 * 2
+    kept_rows = kept * (1 if scored_k else 2) + (kept if (scored_k and reread) else 0)
+    return (cand * hkv * d * 2 + scored_k * hkv * d * 2 + kept_rows * hkv * d * 2
             + hq * d * 2 + hq * d * 4 + hq * 4)
 
 
@@ -698,6 +701,7 @@ def run_gpu(args, rank: int, world: int, dist):
                     f"{B} x 64K sequences",
             "us_per_step": round(hisa_step * 1e3, 2), "queries_per_s": round(B / (hisa_step * 1e-3)),
             "alg_bytes_per_query": hisa_bytes(w.ctx_len),
+            "read_bytes_per_query": hisa_bytes(w.ctx_len, reread=True),
             "GB_s": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9, 1),
             "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4),
             "traffic": (lambda t: None if t is None else t * B // 64)(

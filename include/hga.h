@@ -300,10 +300,12 @@ hga_status hga_prefill_noalloc(const void* q, int32_t n_q_heads, int32_t n_queri
                                const hga_params* p, float* out, cudaStream_t stream);
 
 /*
- * Block-then-token routed decode (the HISA article's two steps: a coarse filter
- * on per-block feature vectors keeps the best blocks, always with the beginning
- * and the end of the text, then token-level scoring runs only inside the kept
- * blocks, taking the indexer's O(L^2) cost to O(L^2/B + L m B)). Blocks are the
+ * Block-then-token routed decode, after the HISA article (shijienb.com news page
+ * on Hierarchical Indexing Sparse Attention): its "step one, block-level coarse
+ * filter" section scores one feature vector per fixed-size block and keeps the
+ * best blocks, always with the beginning and the end of the text, then scores
+ * tokens only inside the kept blocks; its advantages paragraph gives the
+ * indexer cost going from O(L^2) to O(L^2/B + L m B). Blocks are the
  * chunks, with the summaries of hga_build_summaries (only chunk_sum is read),
  * and both steps use the head-summed score of hga_route. Per sequence b and KV
  * head h with nf = seq_lens[b] / chunk full chunks:

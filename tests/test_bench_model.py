@@ -47,7 +47,7 @@ def test_hisa_bytes_match_the_oracles_scoring(L, k_tok):
     inp = synth.decode_inputs(w, lengths=[L], max_len=max(L, 384))
     C, d, hkv, hq = w.chunk, w.head_dim, w.n_kv_heads, w.n_q_heads
     R = hq // hkv
-    total = 0
+    total = reread = 0
     for h in range(hkv):
         K = np.ascontiguousarray(inp.k[0, h, :L])
         cs, _ = oracle.summaries(K, C, w.group)
@@ -56,9 +56,12 @@ def test_hisa_bytes_match_the_oracles_scoring(L, k_tok):
         n_cand = oracle.hisa_candidates(L, C, w.top_chunks)
         n_blocks = scored - n_cand                                   # block summaries scored
         token_rows = n_cand if n_cand > k_tok else 0                 # K rows the token step reads
-        total += (n_blocks + token_rows) * d * 2 + toks.size * d * 2 * 2
+        kept_rows = toks.size if token_rows else 2 * toks.size       # V (K too when no token step ran)
+        total += (n_blocks + token_rows + kept_rows) * d * 2
+        reread += toks.size * d * 2 if token_rows else 0             # kept K read again by the attention
     total += hq * d * 2 + hq * d * 4 + hq * 4
     assert bench.hisa_bytes(L, k_tok) == total
+    assert bench.hisa_bytes(L, k_tok, reread=True) == total + reread
 
 
 def test_prefill_flops_count_every_query_key_pair():
