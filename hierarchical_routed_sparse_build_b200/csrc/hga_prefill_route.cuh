@@ -128,23 +128,42 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
   float* gsc = reinterpret_cast<float*>(smem + lay.gsc);
   int* gstart = reinterpret_cast<int*>(smem + lay.gstart);
 
-  // Head-summed queries of the block (fp32, 16-byte loads of 8 head dims).
+  // Head-summed queries of the block (fp32, 16-byte loads of 8 head dims). Each
+  // thread takes two (query, 8-dim unit) items per pass and issues the loads of all
+  // their heads before summing (heads in ascending order), 16 loads in flight.
   float* qs = reinterpret_cast<float*>(smem + lay.qs);
   const int q0 = blk * a.block;
-  for (int i = tid; i < kBlockQ * (D / 8); i += kRoutedThreads) {
-    const int row = i / (D / 8), u = i - row * (D / 8);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const int qi = q0 + row;
-    if (qi < a.T) {
-      const uint16_t* base = a.q + ((int64_t)qi * a.hq + (int64_t)h * a.R) * D + 8 * u;
-      for (int hh = 0; hh < a.R; ++hh) {
-        const uint4 v = ldg_nc(base + (int64_t)hh * D);
-        acc[0] += bf16_lo(v.x); acc[1] += bf16_hi(v.x); acc[2] += bf16_lo(v.y); acc[3] += bf16_hi(v.y);
-        acc[4] += bf16_lo(v.z); acc[5] += bf16_hi(v.z); acc[6] += bf16_lo(v.w); acc[7] += bf16_hi(v.w);
-      }
+  constexpr int kItems = kBlockQ * (D / 8);
+  for (int i0 = tid; i0 < kItems; i0 += 2 * kRoutedThreads) {
+    uint4 v[2][kMaxHeadsPerKv];
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int i = i0 + s2 * kRoutedThreads;
+      const int row = i / (D / 8), u = i - row * (D / 8);
+      const bool live = i < kItems && q0 + row < a.T;
+      const uint16_t* base = a.q + ((int64_t)(q0 + row) * a.hq + (int64_t)h * a.R) * D + 8 * u;
+#pragma unroll
+      for (int hh = 0; hh < kMaxHeadsPerKv; ++hh)
+        v[s2][hh] = (live && hh < a.R) ? ldg_nc(base + (int64_t)hh * D) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) qs[row * D + 8 * u + c] = acc[c];
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int i = i0 + s2 * kRoutedThreads;
+      const int row = i / (D / 8), u = i - row * (D / 8);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int hh = 0; hh < kMaxHeadsPerKv; ++hh) {
+        if (hh < a.R) {
+          const uint4 w = v[s2][hh];
+          acc[0] += bf16_lo(w.x); acc[1] += bf16_hi(w.x); acc[2] += bf16_lo(w.y); acc[3] += bf16_hi(w.y);
+          acc[4] += bf16_lo(w.z); acc[5] += bf16_hi(w.z); acc[6] += bf16_lo(w.w); acc[7] += bf16_hi(w.w);
+        }
+      }
+      if (i < kItems) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) qs[row * D + 8 * u + c] = acc[c];
+      }
+    }
   }
   __syncthreads();
   // A fragments of the head-summed queries, hi/lo bf16 split, permuted head-dim
