@@ -216,14 +216,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_attn_kernel(const Prefi
     tmem_ld32(tS + lane_off + 0, sv[0]);
     tmem_ld32(tS + lane_off + 32, sv[1]);
     tmem_wait_ld();
-    const bool masked_tile = (j + 1) * kPfKeys > n_cache;
-    if (masked_tile) {
+    // key entry e is attended by this row iff it is a cache entry or an own token
+    // at or before the row's query: e < n_cache + p + 1 (and e < n_keys)
+    const int lim = min(n_cache + p + 1, n_keys) - j * kPfKeys;  // columns c < lim
+    if (lim < kPfKeys) {
 #pragma unroll
-      for (int c = 0; c < kPfKeys; ++c) {
-        const int e = j * kPfKeys + c;
-        const bool valid = e < n_cache || (e < n_keys && (e - n_cache) <= p);
-        if (!valid) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-      }
+      for (int c = 0; c < kPfKeys; ++c)
+        if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
     }
     float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll

@@ -186,3 +186,23 @@ def test_prefill_wait_expiry_is_reported_and_clean(hga, fail_tile):
         for h in range(4):
             ref = pf.oracle_attend(b, h, idx_h[b, h, :n_h[b, h]].astype(np.int64))
             assert_attention_close(out_h[b * 64:(b + 1) * 64, h * 8:(h + 1) * 8], ref, f"after expiry b{b} h{h}")
+
+
+@pytest.mark.parametrize("L0,T,step", [(63488, 2048, 3), (5077, 192, 1)])
+def test_prefill_attend_on_gpu_lists(hga, L0, T, step):
+    # The attention kernel on the lists the GPU routed, against the oracle's
+    # attention over the same list: every (block, KV head) of the ragged case,
+    # every third one at full size (43 of 128, spread over all blocks and heads).
+    w = synth.PREFILL_64K if L0 == 63488 else small(16, 2, L0, T)
+    pf = Prefill(hga, w, L0, T)
+    idx, n = pf.route()
+    no_err(hga)
+    idx_h, n_h = idx.cpu().numpy(), n.cpu().numpy()
+    out = torch.full((T, w.n_q_heads, 128), 7.0, dtype=torch.float32, device="cuda")
+    hga.hga_prefill_attend(pf.q, w.n_q_heads, T, w.block, pf.kv, L0, idx, pf.stride, n, pf.p, out)
+    no_err(hga)
+    out_h = out.cpu().numpy()
+    units = [(b, h) for b in range(pf.nb) for h in range(w.n_kv_heads)][::step]
+    for (b, h) in units:
+        ref = pf.oracle_attend(b, h, idx_h[b, h, :n_h[b, h]].astype(np.int64))
+        assert_attention_close(out_h[b * 64:(b + 1) * 64, h * pf.R:(h + 1) * pf.R], ref, f"b{b} h{h}")
