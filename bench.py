@@ -70,12 +70,14 @@ HISA_SOURCES = DECODE_SOURCES + ("hga_hisa.cuh",)
 HISA_TOKENS = 2048  # tokens kept by the block-then-token decode (below the 2304 the two-level route keeps)
 
 
-def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64, reread: bool = False) -> int:
+def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64, reread: bool = False, logits: bool = False) -> int:
     """Algorithmic HBM bytes of one block-then-token decode query (all KV heads): candidate chunk
     summaries, K of every candidate token (the token step scores them; that covers the kept tokens' K),
     V of the kept tokens (K and V when every candidate is kept, the token step then being skipped), q,
-    out and lse. reread=True adds what the kernel reads beyond that: the kept tokens' K a second time
-    in its attention phase (the token step keeps only head-summed scores)."""
+    out and lse. What the kernels move beyond that: reread=True (hga_decode_hisa) adds the kept tokens'
+    K a second time in the attention phase; logits=True (hga_decode_hisa_ws) adds the workspace
+    traffic instead, the token step writing 8 fp32 logits per candidate and the attention reading
+    those of the kept tokens."""
     C, d, hkv, hq = w.chunk, w.head_dim, w.n_kv_heads, w.n_q_heads
     nf = L // C
     if nf <= 2:
@@ -86,8 +88,9 @@ def hisa_bytes(L: int, k_tok: int = HISA_TOKENS, w=W64, reread: bool = False) ->
     kept = min(k_tok, n_ct)
     scored_k = n_ct if n_ct > k_tok else 0
     kept_rows = kept * (1 if scored_k else 2) + (kept if (scored_k and reread) else 0)
+    lg = (scored_k + kept) * hkv * 8 * 4 if (scored_k and logits) else 0
     return (cand * hkv * d * 2 + scored_k * hkv * d * 2 + kept_rows * hkv * d * 2
-            + hq * d * 2 + hq * d * 4 + hq * 4)
+            + hq * d * 2 + hq * d * 4 + hq * 4 + lg)
 
 
 def kernel_source_hash(names=DECODE_SOURCES) -> str:
@@ -691,17 +694,24 @@ def run_gpu(args, rank: int, world: int, dist):
     # then the top 2048 tokens of their 4352 candidates
     hisa_ms = timed(max(10, args.steps // 2),
                     lambda: cache.decode_hisa(q, HISA_TOKENS, out, lse))
+    reread_ms = timed(max(10, args.steps // 2),
+                      lambda: cache.decode_hisa(q, HISA_TOKENS, out, lse, logits_workspace=False))
     st, bits = hga.hga_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the block-then-token decode: {bits}")
     hisa_step = statistics.median(hisa_ms)
+    reread_step = statistics.median(reread_ms)
     hbm_peak, _ = peaks()
-    hisa = {"what": "hga_decode_hisa: top-32 chunks by summary (plus first and last), then the top "
-                    f"{HISA_TOKENS} of their tokens by the head-summed indexer score, exact attention over them; "
+    hisa = {"what": "hga_decode_hisa_ws: top-32 chunks by summary (plus first and last), then the top "
+                    f"{HISA_TOKENS} of their tokens by the head-summed indexer score (the sum of per-head "
+                    "logits the token step keeps in a workspace), exact attention over them reading only V; "
                     f"{B} x 64K sequences",
             "us_per_step": round(hisa_step * 1e3, 2), "queries_per_s": round(B / (hisa_step * 1e-3)),
             "alg_bytes_per_query": hisa_bytes(w.ctx_len),
-            "read_bytes_per_query": hisa_bytes(w.ctx_len, reread=True),
+            "moved_bytes_per_query": hisa_bytes(w.ctx_len, logits=True),
+            "k_reread": {"what": "hga_decode_hisa (no workspace: the attention reads the kept tokens' K again)",
+                         "us_per_step": round(reread_step * 1e3, 2),
+                         "moved_bytes_per_query": hisa_bytes(w.ctx_len, reread=True)},
             "GB_s": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9, 1),
             "frac_hbm": round(B * hisa_bytes(w.ctx_len) / (hisa_step * 1e-3) / 1e9 / hbm_peak, 4),
             "traffic": (lambda t: None if t is None else t * B // 64)(

@@ -26,7 +26,7 @@ __all__ = [
     "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
     "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
     "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer", "hga_decode_hisa", "hga_max_hisa_tokens",
-    "hga_decode_workspace_size", "hga_decode_ws",
+    "hga_decode_workspace_size", "hga_decode_ws", "hga_decode_hisa_workspace_size", "hga_decode_hisa_ws",
     "HGA_OPT_CTAS_PER_HEAD", "HGA_OPT_DECODE_KERNEL",
     "HGA_OPT_TEST_EXPIRE_PREFILL_WAIT", "STATUS_NAMES",
     "EXPORTED",
@@ -46,7 +46,8 @@ EXPORTED = ("hga_summary_bytes", "hga_build_summaries", "hga_max_routed_tokens",
             "hga_status_string", "hga_route_blocks", "hga_prefill_attend", "hga_prefill_workspace_size",
             "hga_prefill", "hga_prefill_noalloc", "hga_append", "hga_route_blocks_growing",
             "hga_prefill_growing_workspace_size", "hga_prefill_growing", "hga_host_kv_pointer",
-            "hga_decode_hisa", "hga_max_hisa_tokens", "hga_decode_workspace_size", "hga_decode_ws")
+            "hga_decode_hisa", "hga_max_hisa_tokens", "hga_decode_workspace_size", "hga_decode_ws",
+            "hga_decode_hisa_workspace_size", "hga_decode_hisa_ws")
 
 
 class HgaError(RuntimeError):
@@ -102,6 +103,8 @@ def _load() -> ctypes.CDLL:
         "hga_prefill_noalloc": ([vp, i32, i32, i32, KV, i32, vp, vp, P, vp, vp], i32),
         "hga_decode_workspace_size": ([KV, i32, P], sz),
         "hga_decode_ws": ([vp, i32, KV, vp, vp, P, vp, vp, vp, i32, vp, vp, sz, vp], i32),
+        "hga_decode_hisa_workspace_size": ([KV, P], sz),
+        "hga_decode_hisa_ws": ([vp, i32, KV, vp, P, i32, vp, vp, vp, i32, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -291,6 +294,22 @@ def hga_decode_hisa(q, n_q_heads: int, kv: hga_kv, chunk_sum, p: hga_params, top
     _check(_lib.hga_decode_hisa(_addr(q), n_q_heads, ctypes.byref(kv), _addr(chunk_sum), ctypes.byref(p),
                                 top_tokens, _addr(out), _addr(lse), _addr(idx), idx_stride, _addr(n_idx),
                                 _stream(stream)), "hga_decode_hisa")
+
+
+def hga_decode_hisa_workspace_size(kv: hga_kv, p: hga_params) -> int:
+    n = _lib.hga_decode_hisa_workspace_size(ctypes.byref(kv), ctypes.byref(p))
+    if n == 0:
+        raise HgaError(1, "hga_decode_hisa_workspace_size")
+    return int(n)
+
+
+def hga_decode_hisa_ws(q, n_q_heads: int, kv: hga_kv, chunk_sum, p: hga_params, top_tokens: int, out, workspace,
+                       workspace_bytes: int, lse=None, idx=None, idx_stride: int = 0, n_idx=None,
+                       stream=None) -> None:
+    """hga_decode_hisa with a logits workspace: the kept tokens' K is read once."""
+    _check(_lib.hga_decode_hisa_ws(_addr(q), n_q_heads, ctypes.byref(kv), _addr(chunk_sum), ctypes.byref(p),
+                                   top_tokens, _addr(out), _addr(lse), _addr(idx), idx_stride, _addr(n_idx),
+                                   _addr(workspace), workspace_bytes, _stream(stream)), "hga_decode_hisa_ws")
 
 
 def hga_max_hisa_tokens(kv: hga_kv, p: hga_params, top_tokens: int) -> int:

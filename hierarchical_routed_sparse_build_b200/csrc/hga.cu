@@ -566,6 +566,57 @@ int hisa_max_routed(const hga_kv* kv, const hga_params* p, int32_t top_tokens) {
   return most < top_tokens ? most : top_tokens;
 }
 
+
+// Floats of the logits workspace per (sequence, KV head): 8 per candidate of the
+// token step, for the most candidates at any length.
+int64_t hisa_logit_stride(const hga_kv* kv, const hga_params* p) {
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  routing_args(a, kv, p);
+  return (int64_t)hisa_tok_pad(p->chunk, a.kcap) * kMaxHeadsPerKv;
+}
+
+hga_status hisa_impl(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum, const hga_params* p,
+                     int32_t top_tokens, float* out, float* lse, int32_t* idx, int32_t idx_stride, int32_t* n_idx,
+                     float* logits, cudaStream_t stream) {
+  hga_status s = check_kv(kv, true);
+  if (s != HGA_OK) return s;
+  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
+  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
+  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || !aligned16(chunk_sum) || out == nullptr ||
+      top_tokens < 1)
+    return HGA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
+  if (idx != nullptr && idx_stride < hisa_max_routed(kv, p, top_tokens)) return HGA_ERR_INVALID_ARG;
+  if (p->chunk % 16 != 0) return HGA_ERR_UNSUPPORTED;  // token batches of 16 stay inside one chunk
+  RoutedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.kv = make_kv_view(kv);
+  a.sv = make_sum_view(kv, p, chunk_sum, nullptr);
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = n_q_heads;
+  a.R = n_q_heads / kv->n_kv_heads;
+  routing_args(a, kv, p);
+  // never more than the most candidates at any length: a larger top_tokens keeps every candidate
+  // either way, and this bounds the shared-memory list
+  a.k_tok = hisa_max_routed(kv, p, top_tokens);
+  a.scale_log2 = scale_log2(p, kv->head_dim);
+  a.out = out;
+  a.lse = lse;
+  a.idx_out = idx;
+  a.n_idx_out = n_idx;
+  a.idx_stride = idx ? idx_stride : 0;
+  a.logits = logits;
+  a.lg_stride = logits ? hisa_logit_stride(kv, p) : 0;
+  const int smem = HisaSmem(kv->head_dim, a.n_pad, a.kcap, hisa_tok_pad(p->chunk, a.kcap), a.k_tok).total;
+  if (smem > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
+  const int units = kv->batch * kv->n_kv_heads;
+  const int P = pick_cluster(units);
+  cudaError_t e = kv->head_dim == 128 ? launch_hisa<128>(a, units, P, smem, stream)
+                                      : launch_hisa<64>(a, units, P, smem, stream);
+  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace hga
 
@@ -786,40 +837,24 @@ int32_t hga_max_hisa_tokens(const hga_kv* kv, const hga_params* p, int32_t top_t
 hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
                            const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,
                            int32_t idx_stride, int32_t* n_idx, cudaStream_t stream) {
-  hga_status s = check_kv(kv, true);
-  if (s != HGA_OK) return s;
-  if ((s = check_params(p, kv, true)) != HGA_OK) return s;
-  if ((s = check_heads(n_q_heads, kv)) != HGA_OK) return s;
-  if (q == nullptr || !aligned16(q) || chunk_sum == nullptr || !aligned16(chunk_sum) || out == nullptr ||
-      top_tokens < 1)
+  return hisa_impl(q, n_q_heads, kv, chunk_sum, p, top_tokens, out, lse, idx, idx_stride, n_idx, nullptr, stream);
+}
+
+size_t hga_decode_hisa_workspace_size(const hga_kv* kv, const hga_params* p) {
+  if (check_kv(kv, false) != HGA_OK || check_params(p, kv, true) != HGA_OK) return 0;
+  return (size_t)kv->batch * kv->n_kv_heads * (size_t)hisa_logit_stride(kv, p) * sizeof(float);
+}
+
+hga_status hga_decode_hisa_ws(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                              const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,
+                              int32_t idx_stride, int32_t* n_idx, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  const size_t need = hga_decode_hisa_workspace_size(kv, p);
+  if (need == 0) return HGA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
     return HGA_ERR_INVALID_ARG;
-  if ((idx == nullptr) != (n_idx == nullptr)) return HGA_ERR_INVALID_ARG;
-  if (idx != nullptr && idx_stride < hisa_max_routed(kv, p, top_tokens)) return HGA_ERR_INVALID_ARG;
-  if (p->chunk % 16 != 0) return HGA_ERR_UNSUPPORTED;  // token batches of 16 stay inside one chunk
-  RoutedArgs a;
-  std::memset(&a, 0, sizeof a);
-  a.kv = make_kv_view(kv);
-  a.sv = make_sum_view(kv, p, chunk_sum, nullptr);
-  a.q = static_cast<const uint16_t*>(q);
-  a.hq = n_q_heads;
-  a.R = n_q_heads / kv->n_kv_heads;
-  routing_args(a, kv, p);
-  // never more than the most candidates at any length: a larger top_tokens keeps every candidate
-  // either way, and this bounds the shared-memory list
-  a.k_tok = hisa_max_routed(kv, p, top_tokens);
-  a.scale_log2 = scale_log2(p, kv->head_dim);
-  a.out = out;
-  a.lse = lse;
-  a.idx_out = idx;
-  a.n_idx_out = n_idx;
-  a.idx_stride = idx ? idx_stride : 0;
-  const int smem = HisaSmem(kv->head_dim, a.n_pad, a.kcap, hisa_tok_pad(p->chunk, a.kcap), a.k_tok).total;
-  if (smem > kMaxSmemPerCta) return HGA_ERR_UNSUPPORTED;
-  const int units = kv->batch * kv->n_kv_heads;
-  const int P = pick_cluster(units);
-  cudaError_t e = kv->head_dim == 128 ? launch_hisa<128>(a, units, P, smem, stream)
-                                      : launch_hisa<64>(a, units, P, smem, stream);
-  return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA;
+  return hisa_impl(q, n_q_heads, kv, chunk_sum, p, top_tokens, out, lse, idx, idx_stride, n_idx,
+                   static_cast<float*>(workspace), stream);
 }
 
 hga_status hga_route_blocks(const void* q, int32_t n_q_heads, int32_t n_queries, int32_t block,

@@ -118,28 +118,28 @@ __device__ __forceinline__ void store_rows(uint4* tile, const uint4 (&x)[TileGeo
   }
 }
 
-// QK^T of one tile from the shared K copy, then the online-softmax update.
-// Returns the PV B fragments (P^T halves, bf16) in b0, b1. sl = softmax scale *
-// log2(e); entries at or past n_valid are masked.
+// S^T of one tile (raw logits): lane (g, t) gets s[0] = (token g, head 2t),
+// s[1] = (g, 2t+1), s[2] = (g+8, 2t), s[3] = (g+8, 2t+1). ka[j], kb[j] hold unit
+// t + 4j of rows g and g+8 (the K fragment map above).
 template <int D>
-__device__ __forceinline__ void qk_softmax(AttnState<D>& st, const uint4* ktile, int n_valid,
-                                           const uint4* qfrag, float sl, int lane, uint32_t& b0,
-                                           uint32_t& b1) {
-  using G = TileGeom<D>;
-  const int g = lane >> 2;
-  const int t = lane & 3;
-  float s[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ void qk_fragments(float (&s)[4], const uint4 (&ka)[TileGeom<D>::KJ],
+                                             const uint4 (&kb)[TileGeom<D>::KJ], const uint4* qfrag, int lane) {
+  s[0] = s[1] = s[2] = s[3] = 0.f;
 #pragma unroll
-  for (int j = 0; j < G::KJ; ++j) {
-    const int u = t + 4 * j;
-    const uint4 ka = ktile[g * G::U + tile_swz(g, u)];
-    const uint4 kb = ktile[(g + 8) * G::U + tile_swz(g + 8, u)];
+  for (int j = 0; j < TileGeom<D>::KJ; ++j) {
     const uint4 qv = qfrag[j * 32 + lane];
-    mma_16816(s, ka.x, kb.x, ka.y, kb.y, qv.x, qv.y);
-    mma_16816(s, ka.z, kb.z, ka.w, kb.w, qv.z, qv.w);
+    mma_16816(s, ka[j].x, kb[j].x, ka[j].y, kb[j].y, qv.x, qv.y);
+    mma_16816(s, ka[j].z, kb[j].z, ka[j].w, kb[j].w, qv.z, qv.w);
   }
-  // s[0]: token g, head 2t   s[1]: token g, head 2t+1
-  // s[2]: token g+8, head 2t s[3]: token g+8, head 2t+1
+}
+
+// Online-softmax update of one tile's logits s (layout of qk_fragments; entries
+// at or past n_valid are masked). Returns the PV B fragments (P^T halves, bf16)
+// in b0, b1. sl = softmax scale * log2(e).
+template <int D>
+__device__ __forceinline__ void softmax_update(AttnState<D>& st, float (&s)[4], int n_valid, float sl, int lane,
+                                               uint32_t& b0, uint32_t& b1) {
+  const int g = lane >> 2;
   if (g >= n_valid) s[0] = s[1] = -INFINITY;
   if (g + 8 >= n_valid) s[2] = s[3] = -INFINITY;
   float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
@@ -168,6 +168,26 @@ __device__ __forceinline__ void qk_softmax(AttnState<D>& st, const uint4* ktile,
   // P^T halves (tokens 0-7, 8-15) -> PV B fragments (head g, tokens 2t.. / 2t+8..)
   b0 = movmatrix_trans(pack_bf16x2(p0, p1));
   b1 = movmatrix_trans(pack_bf16x2(p2, p3));
+}
+
+// QK^T of one tile from the shared K copy, then the online-softmax update.
+template <int D>
+__device__ __forceinline__ void qk_softmax(AttnState<D>& st, const uint4* ktile, int n_valid,
+                                           const uint4* qfrag, float sl, int lane, uint32_t& b0,
+                                           uint32_t& b1) {
+  using G = TileGeom<D>;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  uint4 ka[G::KJ], kb[G::KJ];
+#pragma unroll
+  for (int j = 0; j < G::KJ; ++j) {
+    const int u = t + 4 * j;
+    ka[j] = ktile[g * G::U + tile_swz(g, u)];
+    kb[j] = ktile[(g + 8) * G::U + tile_swz(g + 8, u)];
+  }
+  float s[4];
+  qk_fragments<D>(s, ka, kb, qfrag, lane);
+  softmax_update<D>(st, s, n_valid, sl, lane, b0, b1);
 }
 
 // O^T += V^T P^T for one tile from the shared V copy.

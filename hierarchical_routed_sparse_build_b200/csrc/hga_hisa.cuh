@@ -20,15 +20,21 @@
 //   T1  the candidate tokens, [0, C) + the kept chunks' tokens + [(nf-1)C, L)
 //       (every token when nf <= 2), are split over the CTAs in batches of 16
 //       consecutive positions and scored the same way from registers; their
-//       64-bit keys (score bits, then lower position) and the score range go
-//       to every CTA
+//       64-bit keys (score bits, then lower candidate index, which orders like
+//       the position) and the score range go to every CTA. With a logits
+//       workspace (hga_decode_hisa_ws) a batch is instead one QK^T MMA tile
+//       (tokens x query heads, K fragments loaded straight from HBM): the score
+//       is the sum of the tile's per-head logits, and the logits are stored
+//       (32 B per candidate) for phase A
 //   --  cluster barrier (skipped, with T1 and T2, when the candidates are no
 //       more than the tokens to keep)
 //   T2  top k_tok tokens (select_top_keys on the score range T1 publishes,
 //       ascending positions), in every CTA
 //   A   exact attention over the kept tokens: 16-token tiles split over the
 //       CTAs and round-robin over the warps (hga_attention.cuh), rows staged
-//       in batches of kEntryBatch entries
+//       in batches of kEntryBatch entries; with the logits workspace the tiles
+//       load the stored logits and gather only V (the kept tokens' K is not
+//       read a second time)
 //   --  warp -> CTA -> cluster softmax combine (finish_attention)
 #pragma once
 
@@ -264,6 +270,42 @@ __device__ __forceinline__ void select_top_keys(const uint64_t* keys, int n, int
     if (keys[i] >= kth && pos < r) sel[pos++] = (int)route_key_id(keys[i]);
 }
 
+// attend_tiles with the logits of every entry already computed: tile t of the
+// staged V rows takes the logits of candidates ents[16t .. 16t+15] from lg
+// ([candidate][8] floats, written earlier in this launch: plain loads) in the
+// S^T fragment layout of qk_fragments, then runs the same softmax update and PV.
+template <int D>
+__device__ __forceinline__ void attend_tiles_logits(AttnState<D>& st, const uint32_t* rows, const int* ents,
+                                                    int n_entries, int tile0, int stride, const uint16_t* V,
+                                                    const float* lg, uint4* tile, float sl, int lane) {
+  const int n_tiles = (n_entries + 15) >> 4;
+  if (tile0 >= n_tiles) return;
+  const int g = lane >> 2, t = lane & 3;
+  auto fetch_logits = [&](int tl, float2& la, float2& lb) {
+    const int ia = min(16 * tl + g, n_entries - 1), ib = min(16 * tl + g + 8, n_entries - 1);
+    la = *reinterpret_cast<const float2*>(lg + (int64_t)ents[ia] * 8 + 2 * t);
+    lb = *reinterpret_cast<const float2*>(lg + (int64_t)ents[ib] * 8 + 2 * t);
+  };
+  uint4 vr[TileGeom<D>::NLD];
+  float2 la, lb;
+  fetch_rows<D>(vr, rows + 16 * tile0, V, lane);
+  fetch_logits(tile0, la, lb);
+  for (int tl = tile0; tl < n_tiles; tl += stride) {
+    const int nt = tl + stride;
+    float s[4] = {la.x, la.y, lb.x, lb.y};
+    store_rows<D>(tile, vr, lane);
+    if (nt < n_tiles) {
+      fetch_rows<D>(vr, rows + 16 * nt, V, lane);
+      fetch_logits(nt, la, lb);
+    }
+    __syncwarp();
+    uint32_t b0, b1;
+    softmax_update<D>(st, s, n_entries - 16 * tl, sl, lane, b0, b1);
+    pv<D>(st, tile, b0, b1, lane);
+    __syncwarp();
+  }
+}
+
 // Most candidate tokens of the token step over every length up to max_len:
 // C + kcap*C + (last block and tail, < 2C), or every token when nf <= 2 (< 3C).
 __host__ __device__ inline int hisa_tok_pad(int C, int kcap) { return (kcap + 3) * C; }
@@ -430,7 +472,19 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
 #pragma unroll
     for (int j = 0; j < 8; ++j) qv[j] = qsum[8 * u + j];
     float smin = __int_as_float(0x7f800000), smax = -__int_as_float(0x7f800000);
-    // issue returns the batch's first position; consume takes it back
+    // key of candidate e: its score, then the lower candidate index first (the
+    // candidates are in ascending position, so this is the lower position)
+    auto emit_key = [&](int e, float score) {
+      const uint64_t key = route_key(score, (uint32_t)e);
+      smin = fminf(smin, score);
+      smax = fmaxf(smax, score);
+      if (P == 1) {
+        tkeys[e] = key;
+      } else {
+        for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(tkeys, pr)[e] = key;
+      }
+    };
+    // issue returns the batch's first position (unused by consume)
     auto issue = [&](int j, uint4(&x)[NLD]) -> int {
       const int bi = bb0 + j;
       const int nv = min(16, n_ct - 16 * bi);
@@ -445,7 +499,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
       }
       return t0;
     };
-    auto consume = [&](int j, const uint4(&x)[NLD], int t0) {
+    auto consume = [&](int j, const uint4(&x)[NLD], int /* first position */) {
       const int bi = bb0 + j;
       float v[NLD];
 #pragma unroll
@@ -453,40 +507,81 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
       int idx;
       const float score = butterfly_sum<NLD>(v, lane, idx);
       const int i = RPI * idx + rsub;
-      if ((lane & 1) == 0 && i < n_ct - 16 * bi) {
-        const uint64_t key = route_key(score, (uint32_t)(t0 + i));
-        smin = fminf(smin, score);
-        smax = fmaxf(smax, score);
-        if (P == 1) {
-          tkeys[16 * bi + i] = key;
-        } else {
-          for (int pr = 0; pr < P; ++pr) cluster.map_shared_rank(tkeys, pr)[16 * bi + i] = key;
+      if ((lane & 1) == 0 && i < n_ct - 16 * bi) emit_key(16 * bi + i, score);
+    };
+    if (a.logits == nullptr) {
+      uint4 xa[NLD], xb[NLD];
+      int ta = 0, tb = 0;
+      if (warp < nb) ta = issue(warp, xa);
+      if (warp + kRoutedWarps < nb) tb = issue(warp + kRoutedWarps, xb);
+      for (int j = warp; j < nb; j += 2 * kRoutedWarps) {
+        consume(j, xa, ta);
+        if (j + 2 * kRoutedWarps < nb) ta = issue(j + 2 * kRoutedWarps, xa);
+        if (j + kRoutedWarps < nb) {
+          consume(j + kRoutedWarps, xb, tb);
+          if (j + 3 * kRoutedWarps < nb) tb = issue(j + 3 * kRoutedWarps, xb);
         }
       }
-    };
-    uint4 xa[NLD], xb[NLD];
-    int ta = 0, tb = 0;
-    if (warp < nb) ta = issue(warp, xa);
-    if (warp + kRoutedWarps < nb) tb = issue(warp + kRoutedWarps, xb);
-    for (int j = warp; j < nb; j += 2 * kRoutedWarps) {
-      consume(j, xa, ta);
-      if (j + 2 * kRoutedWarps < nb) ta = issue(j + 2 * kRoutedWarps, xa);
-      if (j + kRoutedWarps < nb) {
-        consume(j + kRoutedWarps, xb, tb);
-        if (j + 3 * kRoutedWarps < nb) tb = issue(j + 3 * kRoutedWarps, xb);
+    } else {
+      // QK^T tiles: lane (g, t) loads unit t + 4j of the batch's rows g and g+8
+      // (64 contiguous bytes of each row per warp instruction); the score of a
+      // token is the sum over the query heads of its logits (padding heads have
+      // zero queries), reduced over the four lanes that share the token
+      constexpr int KJ = TG::KJ;
+      float* lg = a.logits + (int64_t)unit * a.lg_stride;
+      const int gq = lane >> 2, tq = lane & 3;
+      auto issue_mma = [&](int j, uint4(&ka)[KJ], uint4(&kb)[KJ]) {
+        const int bi = bb0 + j;
+        const int nv = min(16, n_ct - 16 * bi);
+        const uint16_t* src = a.kv.k + (int64_t)tok_row(batch_tok(bi)) * D + 8 * tq;
+        const int ra = min(gq, nv - 1), rb = min(gq + 8, nv - 1);
+#pragma unroll
+        for (int jj = 0; jj < KJ; ++jj) {
+          ka[jj] = ldg_stream(src + (int64_t)ra * D + 32 * jj);
+          kb[jj] = ldg_stream(src + (int64_t)rb * D + 32 * jj);
+        }
+      };
+      auto consume_mma = [&](int j, const uint4(&ka)[KJ], const uint4(&kb)[KJ]) {
+        const int bi = bb0 + j;
+        const int nv = min(16, n_ct - 16 * bi);
+        float sv[4];
+        qk_fragments<D>(sv, ka, kb, qfrag, lane);
+        float sa = sv[0] + sv[1], sb = sv[2] + sv[3];
+        sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
+        sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
+        sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 2);
+        sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 2);
+        const int ea = 16 * bi + gq, eb = ea + 8;
+        if (gq < nv) *reinterpret_cast<float2*>(lg + (int64_t)ea * 8 + 2 * tq) = make_float2(sv[0], sv[1]);
+        if (gq + 8 < nv) *reinterpret_cast<float2*>(lg + (int64_t)eb * 8 + 2 * tq) = make_float2(sv[2], sv[3]);
+        if (tq == 0) {
+          if (gq < nv) emit_key(ea, sa);
+          if (gq + 8 < nv) emit_key(eb, sb);
+        }
+      };
+      uint4 ka0[KJ], kb0[KJ], ka1[KJ], kb1[KJ];
+      if (warp < nb) issue_mma(warp, ka0, kb0);
+      if (warp + kRoutedWarps < nb) issue_mma(warp + kRoutedWarps, ka1, kb1);
+      for (int j = warp; j < nb; j += 2 * kRoutedWarps) {
+        consume_mma(j, ka0, kb0);
+        if (j + 2 * kRoutedWarps < nb) issue_mma(j + 2 * kRoutedWarps, ka0, kb0);
+        if (j + kRoutedWarps < nb) {
+          consume_mma(j + kRoutedWarps, ka1, kb1);
+          if (j + 3 * kRoutedWarps < nb) issue_mma(j + 3 * kRoutedWarps, ka1, kb1);
+        }
       }
     }
     publish_range(smin, smax, tmm, kTmmTok, cluster, P, cr);
     cluster.sync();
     float lo, hi;
     cluster_range(tmm, kTmmTok, P, lo, hi);
-    // top k_tok of the n_ct keys; candidates are in ascending position, so the
-    // ordered compaction writes the kept positions ascending
+    // top k_tok of the n_ct keys, as candidate indices in ascending order (so
+    // the kept positions come out ascending)
     select_top_keys(tkeys, n_ct, k_tok, lo, hi, tsel, hist, misc, scratch, kred);
     __syncthreads();
   }
   const int S = keep_all ? n_ct : k_tok;
-  auto entry_tok = [&](int e) -> int { return keep_all ? cand_tok(e) : tsel[e]; };
+  auto entry_tok = [&](int e) -> int { return cand_tok(keep_all ? e : tsel[e]); };
 
   // ------------------------------------------------------------------- A
   const int n_tiles = (S + 15) / 16;
@@ -508,7 +603,11 @@ __global__ void __launch_bounds__(kRoutedThreads, 2) hisa_decode_kernel(const Ro
     // padding entries of the last tile read the batch's first row (masked)
     for (int i = tid; i < n_t * 16; i += kRoutedThreads) rows[i] = tok_row(entry_tok(eb + (i < n_e ? i : 0)));
     __syncthreads();
-    attend_tiles<D>(st, rows, n_e, warp, kRoutedWarps, a.kv.k, a.kv.v, qfrag, tile, a.scale_log2, lane);
+    if (a.logits != nullptr && !keep_all)
+      attend_tiles_logits<D>(st, rows, tsel + eb, n_e, warp, kRoutedWarps, a.kv.v,
+                             a.logits + (int64_t)unit * a.lg_stride, tile, a.scale_log2, lane);
+    else
+      attend_tiles<D>(st, rows, n_e, warp, kRoutedWarps, a.kv.k, a.kv.v, qfrag, tile, a.scale_log2, lane);
   }
   finish_attention<D>(st, a, cluster, P, cr, b, h, red_o, red_m, red_l, cta_o, cta_m, cta_l);
 }

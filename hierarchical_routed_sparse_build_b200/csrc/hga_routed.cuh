@@ -74,6 +74,9 @@ struct RoutedArgs {
   const int32_t* idx_in;
   const int32_t* n_idx_in;
   int idx_stride;
+  float* logits;      // block-then-token decode: per-head logits of the token step's candidates,
+                      // [B * Hkv][lg_stride / 8][8] (null: the attention recomputes them from K)
+  int64_t lg_stride;  // floats per (sequence, KV head)
 };
 
 // Shared-memory carve-up (byte offsets), identical on host and device. One

@@ -9,7 +9,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (hga_append, hga_attend, hga_build_summaries, hga_decode_hisa, hga_decode_workspace_size, hga_decode_ws,
+from . import (hga_append, hga_attend, hga_build_summaries, hga_decode_hisa, hga_decode_hisa_workspace_size,
+               hga_decode_hisa_ws, hga_decode_workspace_size, hga_decode_ws,
                hga_max_hisa_tokens, hga_max_routed_tokens, hga_route, hga_summary_bytes, make_kv, make_params)
 
 
@@ -83,8 +84,12 @@ class RoutedCache:
     def build_summaries(self, stream=None) -> None:
         hga_build_summaries(self.kv, self.params, self.chunk_sum, self.group_sum, stream)
 
-    def decode_hisa(self, q, top_tokens: int, out=None, lse=None, want_idx: bool = False, stream=None):
-        """Block-then-token routed decode (top chunks by summary, then the top_tokens tokens inside them)."""
+    def decode_hisa(self, q, top_tokens: int, out=None, lse=None, want_idx: bool = False, stream=None,
+                    logits_workspace: bool = True):
+        """Block-then-token routed decode (top chunks by summary, then the top_tokens tokens inside them).
+        With logits_workspace (the default) the token step keeps its per-head logits in a workspace owned by
+        this cache and the attention reads only V for the kept tokens (hga_decode_hisa_ws); without it the
+        attention re-reads their K (hga_decode_hisa)."""
         q = self.q_tensor(q)
         if out is None:
             out, lse = self.out_buffers()
@@ -95,8 +100,16 @@ class RoutedCache:
             idx = torch.full((self.batch, self.n_kv_heads, max(stride, 1)), -1, dtype=torch.int32,
                              device=self.device)
             n_idx = torch.zeros((self.batch, self.n_kv_heads), dtype=torch.int32, device=self.device)
-        hga_decode_hisa(q, self.n_q_heads, self.kv, self.chunk_sum, self.params, top_tokens, out, lse, idx,
-                        max(stride, 1) if want_idx else 0, n_idx, stream)
+        if logits_workspace:
+            if getattr(self, "hisa_workspace", None) is None:
+                self.hisa_ws_bytes = hga_decode_hisa_workspace_size(self.kv, self.params)
+                self.hisa_workspace = torch.empty(self.hisa_ws_bytes, dtype=torch.uint8, device=self.device)
+            hga_decode_hisa_ws(q, self.n_q_heads, self.kv, self.chunk_sum, self.params, top_tokens, out,
+                               self.hisa_workspace, self.hisa_ws_bytes, lse, idx,
+                               max(stride, 1) if want_idx else 0, n_idx, stream)
+        else:
+            hga_decode_hisa(q, self.n_q_heads, self.kv, self.chunk_sum, self.params, top_tokens, out, lse, idx,
+                            max(stride, 1) if want_idx else 0, n_idx, stream)
         return (out, lse, idx, n_idx) if want_idx else (out, lse)
 
     def append(self, k_new, v_new, stream=None) -> None:

@@ -332,6 +332,30 @@ hga_status hga_decode_hisa(const void* q, int32_t n_q_heads, const hga_kv* kv, c
 int32_t hga_max_hisa_tokens(const hga_kv* kv, const hga_params* p, int32_t top_tokens);
 
 /*
+ * hga_decode_hisa with a caller-owned workspace (device memory, 256-byte
+ * aligned, at least hga_decode_hisa_workspace_size bytes, used by this call
+ * only). The token step then computes the per-head logits q_i . K_t of every
+ * candidate with tensor-core tiles, keeps them in the workspace (fp32,
+ * 32 bytes per candidate), takes tau_t as their sum over the query heads, and
+ * the attention over the kept tokens reads those logits and the kept V rows,
+ * not the kept K rows a second time. Same routing definition and outputs as
+ * hga_decode_hisa (tau_t is summed in another order, which can change the
+ * kept set only between near-equal scores). HGA_ERR_INVALID_ARG for a missing,
+ * misaligned or short workspace; otherwise as hga_decode_hisa.
+ */
+hga_status hga_decode_hisa_ws(const void* q, int32_t n_q_heads, const hga_kv* kv, const void* chunk_sum,
+                              const hga_params* p, int32_t top_tokens, float* out, float* lse, int32_t* idx,
+                              int32_t idx_stride, int32_t* n_idx, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/*
+ * Workspace bytes of hga_decode_hisa_ws: batch * n_kv_heads * 32 bytes per
+ * candidate of the longest context ((min(top_chunks, max_len / chunk - 2) + 3)
+ * * chunk candidates). 0 on invalid arguments.
+ */
+size_t hga_decode_hisa_workspace_size(const hga_kv* kv, const hga_params* p);
+
+/*
  * Growing-history chunked prefill: the same calls as hga_route_blocks /
  * hga_prefill / hga_prefill_workspace_size, except that block b (queries at
  * P_b = cache_len + b * block .. P_b + block - 1) routes over everything before

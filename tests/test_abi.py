@@ -245,3 +245,25 @@ def test_decode_workspace_size_and_validation():
     assert raw_decode_ws(kv, p, ws=FAKE + 16) == INVALID             # not 256-byte aligned
     assert raw_decode_ws(kv, p, nbytes=n - 1) == INVALID             # too small
     assert raw_decode_ws(kv_desc(head_dim=96), p) == UNSUPPORTED     # the decode's own checks still apply
+
+
+def raw_hisa_ws(kv, p, ws=FAKE, nbytes=1 << 30, hq=32, top_tokens=2048):
+    return hga._lib.hga_decode_hisa_ws(FAKE, hq, ctypes.byref(kv), FAKE, ctypes.byref(p), top_tokens, FAKE, None,
+                                       None, 0, None, ws, nbytes, None)
+
+
+def test_hisa_logits_workspace_size_and_validation():
+    kv, p = kv_desc(batch=64), params()
+    n = hga.hga_decode_hisa_workspace_size(kv, p)
+    # 32 bytes (8 fp32 logits) per candidate of the longest context, per (sequence, KV head):
+    # (top_chunks + 3) chunks of candidates, the bound of the token keys
+    nf = kv.max_len // p.chunk
+    assert n == 64 * 4 * (min(p.top_chunks, nf - 2) + 3) * p.chunk * 32
+    assert n >= 64 * 4 * 32 * max(oracle.hisa_candidates(L, p.chunk, p.top_chunks)
+                                  for L in range(kv.max_len - 2 * p.chunk, kv.max_len + 1))
+    assert hga._lib.hga_decode_hisa_workspace_size(ctypes.byref(kv_desc(head_dim=96)), ctypes.byref(p)) == 0
+    assert raw_hisa_ws(kv, p, ws=0) == INVALID                   # no workspace
+    assert raw_hisa_ws(kv, p, ws=FAKE + 16) == INVALID           # not 256-byte aligned
+    assert raw_hisa_ws(kv, p, nbytes=n - 1) == INVALID           # too small
+    assert raw_hisa_ws(kv, p, top_tokens=0) == INVALID           # the block-then-token checks still apply
+    assert raw_hisa_ws(kv, p, hq=48) == UNSUPPORTED

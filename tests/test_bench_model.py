@@ -47,7 +47,7 @@ def test_hisa_bytes_match_the_oracles_scoring(L, k_tok):
     inp = synth.decode_inputs(w, lengths=[L], max_len=max(L, 384))
     C, d, hkv, hq = w.chunk, w.head_dim, w.n_kv_heads, w.n_q_heads
     R = hq // hkv
-    total = reread = 0
+    total = reread = logit_bytes = 0
     for h in range(hkv):
         K = np.ascontiguousarray(inp.k[0, h, :L])
         cs, _ = oracle.summaries(K, C, w.group)
@@ -59,9 +59,12 @@ def test_hisa_bytes_match_the_oracles_scoring(L, k_tok):
         kept_rows = toks.size if token_rows else 2 * toks.size       # V (K too when no token step ran)
         total += (n_blocks + token_rows + kept_rows) * d * 2
         reread += toks.size * d * 2 if token_rows else 0             # kept K read again by the attention
+        # or: 8 fp32 logits written per candidate, read back for the kept tokens
+        logit_bytes += (n_cand + toks.size) * 8 * 4 if token_rows else 0
     total += hq * d * 2 + hq * d * 4 + hq * 4
     assert bench.hisa_bytes(L, k_tok) == total
     assert bench.hisa_bytes(L, k_tok, reread=True) == total + reread
+    assert bench.hisa_bytes(L, k_tok, logits=True) == total + logit_bytes
 
 
 def test_prefill_flops_count_every_query_key_pair():

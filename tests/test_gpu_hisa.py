@@ -22,7 +22,13 @@ def hga():
     return m
 
 
-def run_hisa(hga, w, inp, m, k_tok, units=None, page_table=None, k_pool=None, v_pool=None):
+@pytest.fixture(params=[True, False], ids=["logits_workspace", "k_reread"])
+def logits(request):
+    """hga_decode_hisa_ws (per-head logits kept from the token step) or hga_decode_hisa (K read again)."""
+    return request.param
+
+
+def run_hisa(hga, w, inp, m, k_tok, units=None, page_table=None, k_pool=None, v_pool=None, logits=True):
     from hierarchical_routed_sparse_build_b200.runtime import RoutedCache
     if page_table is None:
         c = RoutedCache(inp.k, inp.v, inp.seq_lens, chunk=w.chunk, group=w.group, top_chunks=m,
@@ -31,7 +37,7 @@ def run_hisa(hga, w, inp, m, k_tok, units=None, page_table=None, k_pool=None, v_
         c = RoutedCache(k_pool, v_pool, inp.seq_lens, chunk=w.chunk, group=w.group, top_chunks=m,
                         top_groups=w.top_groups, n_q_heads=w.n_q_heads, page_table=page_table)
     c.build_summaries()
-    out, lse, idx, n_idx = c.decode_hisa(c.q_tensor(inp.q), k_tok, want_idx=True)
+    out, lse, idx, n_idx = c.decode_hisa(c.q_tensor(inp.q), k_tok, want_idx=True, logits_workspace=logits)
     st, b = hga.hga_get_device_error()
     assert st == 0, b
     R = w.n_q_heads // w.n_kv_heads
@@ -53,41 +59,41 @@ def run_hisa(hga, w, inp, m, k_tok, units=None, page_table=None, k_pool=None, v_
     return exact, len(units)
 
 
-def test_hisa_decode_16k(hga):
+def test_hisa_decode_16k(hga, logits):
     w = synth.DECODE_16K
     inp = synth.decode_inputs(w)
-    exact, n = run_hisa(hga, w, inp, m=16, k_tok=1024)
+    exact, n = run_hisa(hga, w, inp, m=16, k_tok=1024, logits=logits)
     assert exact >= n - 1
 
 
 @pytest.mark.parametrize("ctas", [1, 3, 8])
-def test_hisa_cluster_sizes(hga, ctas):
+def test_hisa_cluster_sizes(hga, ctas, logits):
     w = synth.with_len(synth.DECODE_64K, 12000)
     inp = synth.decode_inputs(w, lengths=[12000, 9999], max_len=12032)
     hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, ctas)
     try:
-        exact, n = run_hisa(hga, w, inp, m=8, k_tok=700)
+        exact, n = run_hisa(hga, w, inp, m=8, k_tok=700, logits=logits)
     finally:
         hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
     assert exact >= n - 1
 
 
-def test_hisa_edge_lengths(hga):
+def test_hisa_edge_lengths(hga, logits):
     # empty, dense (< 3 chunks), candidates fewer than the tokens to keep, ragged tails
     w = synth.Workload("hisa_edge", 1, 32, 4, 128, 0, 128, 16, 4, 2, -1, 31)
     lens = [0, 1, 200, 383, 384, 700, 1000, 2049, 5000]
     inp = synth.decode_inputs(w, lengths=lens, max_len=5120)
-    run_hisa(hga, w, inp, m=4, k_tok=300)
+    run_hisa(hga, w, inp, m=4, k_tok=300, logits=logits)
 
 
 @pytest.mark.parametrize("hq,hkv,d", [(8, 1, 64), (12, 4, 64), (6, 2, 128)])
-def test_hisa_head_shapes(hga, hq, hkv, d):
+def test_hisa_head_shapes(hga, hq, hkv, d, logits):
     w = synth.Workload(f"hisa{hq}x{hkv}x{d}", 1, hq, hkv, d, 4000, 64, 16, 6, 2, -1, 37)
     inp = synth.decode_inputs(w, lengths=[4000, 3333], max_len=4032)
-    run_hisa(hga, w, inp, m=6, k_tok=256)
+    run_hisa(hga, w, inp, m=6, k_tok=256, logits=logits)
 
 
-def test_hisa_paged(hga):
+def test_hisa_paged(hga, logits):
     w = synth.Workload("hisa_paged", 1, 32, 4, 128, 9000, 128, 16, 8, 2, -1, 41)
     lens = np.array([9000, 4100, 6400], dtype=np.int32)
     inp = synth.decode_inputs(w, lengths=list(lens), max_len=9088)
@@ -98,7 +104,7 @@ def test_hisa_paged(hga):
     for b in range(3):
         kpool[table[b]] = inp.k[b].reshape(4, per, 128, 128).transpose(1, 0, 2, 3)
         vpool[table[b]] = inp.v[b].reshape(4, per, 128, 128).transpose(1, 0, 2, 3)
-    exact, n = run_hisa(hga, w, inp, m=8, k_tok=1024, page_table=table, k_pool=kpool, v_pool=vpool)
+    exact, n = run_hisa(hga, w, inp, m=8, k_tok=1024, page_table=table, k_pool=kpool, v_pool=vpool, logits=logits)
     assert exact >= n - 1
 
 
@@ -117,15 +123,15 @@ def test_hisa_full_coverage_is_dense_attention(hga):
             assert_attention_close(out[b, h * 8:(h + 1) * 8].cpu().numpy(), ref, f"dense b{b} h{h}")
 
 
-def test_hisa_decode_64k_sampled(hga):
+def test_hisa_decode_64k_sampled(hga, logits):
     w = synth.DECODE_64K
     inp = synth.decode_inputs(w, lengths=[w.ctx_len] * 2)
-    exact, n = run_hisa(hga, w, inp, m=32, k_tok=2048, units=[(0, 0), (0, 3), (1, 1)])
+    exact, n = run_hisa(hga, w, inp, m=32, k_tok=2048, units=[(0, 0), (0, 3), (1, 1)], logits=logits)
     assert exact >= n - 1
 
 
 @pytest.mark.parametrize("ctas", [0, 3])
-def test_hisa_ties_take_lower_positions(hga, ctas):
+def test_hisa_ties_take_lower_positions(hga, ctas, logits):
     # every key equal: all chunk summaries and all token scores tie, so the kept
     # set is the first k_tok candidates by position (the select's refinement path)
     w = synth.Workload("hisa_ties", 1, 32, 4, 128, 9000, 128, 16, 8, 2, -1, 47)
@@ -136,7 +142,7 @@ def test_hisa_ties_take_lower_positions(hga, ctas):
         from hierarchical_routed_sparse_build_b200.runtime import RoutedCache
         c = RoutedCache(inp.k, inp.v, inp.seq_lens, chunk=128, group=16, top_chunks=8, top_groups=2, n_q_heads=32)
         c.build_summaries()
-        out, _, idx, n_idx = c.decode_hisa(c.q_tensor(inp.q), 700, want_idx=True)
+        out, _, idx, n_idx = c.decode_hisa(c.q_tensor(inp.q), 700, want_idx=True, logits_workspace=logits)
         assert hga.hga_get_device_error()[0] == 0
     finally:
         hga.hga_set_launch_option(hga.HGA_OPT_CTAS_PER_HEAD, 0)
@@ -151,9 +157,9 @@ def test_hisa_ties_take_lower_positions(hga, ctas):
             assert np.array_equal(idx[b, h, :700].cpu().numpy(), ref), f"ties b{b} h{h}"
 
 
-def test_hisa_many_blocks(hga):
+def test_hisa_many_blocks(hga, logits):
     # 64 kept chunks of 126 at 16K: 8448 candidate tokens in shared memory
     w = synth.DECODE_16K
     inp = synth.decode_inputs(w, lengths=[w.ctx_len] * 2)
-    exact, n = run_hisa(hga, w, inp, m=64, k_tok=3000, units=[(0, 0), (0, 2), (1, 3)])
+    exact, n = run_hisa(hga, w, inp, m=64, k_tok=3000, units=[(0, 0), (0, 2), (1, 3)], logits=logits)
     assert exact >= n - 1
