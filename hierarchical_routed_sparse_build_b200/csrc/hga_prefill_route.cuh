@@ -67,40 +67,48 @@ __device__ __forceinline__ void load_b_units(const uint16_t* my_row, int lane, u
   for (int j = 0; j < 4; ++j) bu[j] = ldg_nc(my_row + 8 * (t + 4 * j));
 }
 
-__device__ __forceinline__ void block_scores_tile(const uint4* afrag, const uint4 (&bu)[4], int lane,
-                                                  float& c0max, float& c1max) {
-  float acc[4][4];
+// Two row tiles per call: each A fragment read from shared memory feeds both
+// tiles' MMAs (the fragments are the scan's shared-memory bandwidth). Every
+// (m tile, row tile) accumulator sees the same MMA order as a one-tile scan.
+__device__ __forceinline__ void block_scores_tile2(const uint4* afrag, const uint4 (&bu)[2][4], int lane,
+                                                   float (&cmax)[2][2]) {
+  float acc[2][4][4];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-#pragma unroll 2
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[u][mt][i] = 0.f;
+#pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const int j = ks >> 1, p = ks & 1;
-    const uint32_t b0 = p ? bu[j].z : bu[j].x;
-    const uint32_t b1 = p ? bu[j].w : bu[j].y;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
       for (int hl = 0; hl < 2; ++hl) {
         const uint4 a = afrag[((mt * 8 + ks) * 2 + hl) * 32 + lane];
-        mma_16816(acc[mt], a.x, a.y, a.z, a.w, b0, b1);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          mma_16816(acc[u][mt], a.x, a.y, a.z, a.w, p ? bu[u][j].z : bu[u][j].x, p ? bu[u][j].w : bu[u][j].y);
       }
     }
   }
-  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    m0 = fmaxf(m0, fmaxf(acc[mt][0], acc[mt][2]));
-    m1 = fmaxf(m1, fmaxf(acc[mt][1], acc[mt][3]));
-  }
+  for (int u = 0; u < 2; ++u) {
+    float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, off));
-    m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, off));
+    for (int mt = 0; mt < 4; ++mt) {
+      m0 = fmaxf(m0, fmaxf(acc[u][mt][0], acc[u][mt][2]));
+      m1 = fmaxf(m1, fmaxf(acc[u][mt][1], acc[u][mt][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, off));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, off));
+    }
+    cmax[u][0] = m0;
+    cmax[u][1] = m1;
   }
-  c0max = m0;
-  c1max = m1;
 }
 
 __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const BlockRouteArgs a) {
@@ -198,23 +206,36 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
 
   const uint16_t* cs = a.chunk_sum + (int64_t)h * a.max_chunks * D;
   const uint16_t* gs = a.group_sum + (int64_t)h * a.max_chunks * gpc * D;
-  // chunk scores, 8 candidates per warp tile
+  // chunk scores, 8 candidates per row tile, two row tiles per warp step
   if (n_cand > r) {
     const int n_tiles = (n_cand + 7) / 8;
+    const int n_pairs = (n_tiles + 1) / 2;
+    // rows past the last candidate repeat it (its scores are not stored)
     auto row_of = [&](int tile) { return cs + (int64_t)(min(tile * 8 + (lane >> 2), n_cand - 1) + 1) * D; };
-    uint4 bu[4], bn[4];
-    if (warp < n_tiles) load_b_units(row_of(warp), lane, bu);
-    for (int tile = warp; tile < n_tiles; tile += W) {
-      if (tile + W < n_tiles) load_b_units(row_of(tile + W), lane, bn);
-      float m0, m1;
-      block_scores_tile(afrag, bu, lane, m0, m1);
+    uint4 bu[2][4], bn[2][4];
+    if (warp < n_pairs) {
+      load_b_units(row_of(2 * warp), lane, bu[0]);
+      load_b_units(row_of(2 * warp + 1), lane, bu[1]);
+    }
+    for (int pt = warp; pt < n_pairs; pt += W) {
+      if (pt + W < n_pairs) {
+        load_b_units(row_of(2 * (pt + W)), lane, bn[0]);
+        load_b_units(row_of(2 * (pt + W) + 1), lane, bn[1]);
+      }
+      float cmax[2][2];
+      block_scores_tile2(afrag, bu, lane, cmax);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bu[j] = bn[j];
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bu[u][j] = bn[u][j];
       if ((lane >> 2) == 0) {
         const int t4 = lane & 3;
-        const int ca = tile * 8 + 2 * t4, cb = ca + 1;
-        if (ca < n_cand) keys[ca] = route_key(m0, (uint32_t)(ca + 1));
-        if (cb < n_cand) keys[cb] = route_key(m1, (uint32_t)(cb + 1));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int ca = (2 * pt + u) * 8 + 2 * t4, cb = ca + 1;
+          if (ca < n_cand) keys[ca] = route_key(cmax[u][0], (uint32_t)(ca + 1));
+          if (cb < n_cand) keys[cb] = route_key(cmax[u][1], (uint32_t)(cb + 1));
+        }
       }
     }
     __syncthreads();
@@ -234,20 +255,36 @@ __global__ void __launch_bounds__(kRoutedThreads) block_route_kernel(const Block
       return gs + ((int64_t)sel[ci] * gpc + min(part * 8 + (lane >> 2), gpc - 1)) * D;
     };
     const int n_gt = r * tiles_per_chunk;
-    uint4 bu[4], bn[4];
-    if (warp < n_gt) load_b_units(grow_of(warp), lane, bu);
-    for (int wt = warp; wt < n_gt; wt += W) {
-      const int ci = wt / tiles_per_chunk, part = wt - ci * tiles_per_chunk;
-      if (wt + W < n_gt) load_b_units(grow_of(wt + W), lane, bn);
-      float m0, m1;
-      block_scores_tile(afrag, bu, lane, m0, m1);
+    const int n_pairs = (n_gt + 1) / 2;
+    // tiles past the last repeat it (their scores are not stored)
+    auto grow_at = [&](int wt) { return grow_of(min(wt, n_gt - 1)); };
+    uint4 bu[2][4], bn[2][4];
+    if (warp < n_pairs) {
+      load_b_units(grow_at(2 * warp), lane, bu[0]);
+      load_b_units(grow_at(2 * warp + 1), lane, bu[1]);
+    }
+    for (int pt = warp; pt < n_pairs; pt += W) {
+      if (pt + W < n_pairs) {
+        load_b_units(grow_at(2 * (pt + W)), lane, bn[0]);
+        load_b_units(grow_at(2 * (pt + W) + 1), lane, bn[1]);
+      }
+      float cmax[2][2];
+      block_scores_tile2(afrag, bu, lane, cmax);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bu[j] = bn[j];
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bu[u][j] = bn[u][j];
       if ((lane >> 2) == 0) {
         const int t4 = lane & 3;
-        const int ja = part * 8 + 2 * t4, jb = ja + 1;
-        if (ja < gpc) gsc[ci * gpc + ja] = m0;
-        if (jb < gpc) gsc[ci * gpc + jb] = m1;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int wt = 2 * pt + u;
+          if (wt >= n_gt) continue;
+          const int ci = wt / tiles_per_chunk, part = wt - ci * tiles_per_chunk;
+          const int ja = part * 8 + 2 * t4, jb = ja + 1;
+          if (ja < gpc) gsc[ci * gpc + ja] = cmax[u][0];
+          if (jb < gpc) gsc[ci * gpc + jb] = cmax[u][1];
+        }
       }
     }
     for (int i = tid; i < r; i += kRoutedThreads) gmask[i] = 0u;
